@@ -1,0 +1,16 @@
+"""fp64 CPU oracle for exact attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference legs may import this package.  The product path never does.
+"""
+
+from .attention import (  # noqa: F401
+    attention_forward,
+    attention_head,
+    attention_rows,
+    attention_scores,
+    gather_paged_kv,
+    gqa_kv_head,
+    paged_decode,
+    softmax_with_lse,
+)

@@ -1,0 +1,205 @@
+"""Plain, slow, fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code, table or helper with the CUDA path.
+
+What it computes, and where the pages define it
+-----------------------------------------------
+"Fast Attention Kernels and Operator Fusion" (wpnews.pro), section
+"FlashAttention-Style Kernels", gives the operation as
+
+    Attention(Q, K, V) = softmax(Q K^T / sqrt(d) + M) V
+
+with M an additive mask; its SDPA example uses ``is_causal=True``, i.e. M is
+-inf above the diagonal.  "Kernel Fusion and Custom Kernels" (ai.zenoagi.com),
+section 5 "Intra-Attention Fusion", spells the unfused chain out as
+S = Q K^T -> P = softmax(S) -> O = P V with S and P full N x N matrices; this
+module does exactly that, materialising S and P per head, in float64.  The
+anylearn.cc lesson ("Five things", third point) states that the fused method
+is exact rather than approximate, so the plain definition is the oracle for
+the fused kernel (up to rounding order).
+
+Readings where the pages are silent (each is restated where it is used):
+
+* scale: passed in (1/sqrt(d) in every workload) and multiplied into the
+  scores before the mask is added.
+* causal alignment: query i sees key j iff j <= i (Nq == Nk, so top-left and
+  bottom-right alignment agree and no row is empty).
+* LSE: the natural log of sum_j exp(scale * q_i . k_j) over the visible keys.
+* GQA: query head h uses key/value head h // (Hq // Hkv) (consecutive query
+  heads share one KV head).
+* paged KV: pool layout [num_pages, page_size, Hkv, d]; logical token t of a
+  sequence lives in physical page block_table[t // page_size], slot
+  t % page_size ("Paged Attention Kernels" section and its block-table figure,
+  logical blocks 0,1,2,3 -> physical 17,4,29,8).  Decode has one query per
+  sequence that sees all seq_len cached keys.
+
+Pins (all in ``tests/test_oracle.py``): rows of P sum to one; constant V rows
+are returned unchanged; K == 0 gives the prefix mean of V and LSE = log(count);
+causal row 0 returns v_0 with LSE = scale q_0 . k_0; a pure-Python ``math.fsum``
+brute force on tiny inputs; PyTorch's fp64 CPU ``scaled_dot_product_attention``
+and ``logsumexp`` as a library special case; the pages' block-table example;
+paged gather equal to contiguous KV bit for bit.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "gqa_kv_head",
+    "attention_scores",
+    "softmax_with_lse",
+    "attention_head",
+    "attention_forward",
+    "attention_rows",
+    "gather_paged_kv",
+    "paged_decode",
+]
+
+
+def _f64(x) -> np.ndarray:
+    """Return ``x`` as a float64 ndarray (exact for bf16/fp16/fp32 inputs)."""
+    return np.asarray(x, dtype=np.float64)
+
+
+def gqa_kv_head(h_q: int, Hq: int, Hkv: int) -> int:
+    """KV head read by query head ``h_q``: floor(h_q / (Hq / Hkv)).
+
+    The pages do not mention grouped-query attention; this is the reading in
+    which consecutive query heads share a KV head.
+    """
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return h_q // (Hq // Hkv)
+
+
+def attention_scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
+                     row_offset: int = 0) -> np.ndarray:
+    """S = scale * q k^T + M for one head.
+
+    ``q`` holds query rows ``row_offset .. row_offset + len(q) - 1`` of the head;
+    ``k`` holds all keys.  With ``causal`` the additive mask M is -inf where the
+    key index exceeds the query index ("FlashAttention-Style Kernels",
+    equation with M and the ``is_causal=True`` example).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    s = float(scale) * (q @ k.T)
+    if causal:
+        rows = np.arange(row_offset, row_offset + q.shape[0])[:, None]
+        cols = np.arange(k.shape[0])[None, :]
+        s = np.where(cols > rows, -np.inf, s)
+    return s
+
+
+def softmax_with_lse(s: np.ndarray):
+    """Row softmax of ``s`` and its natural-log log-sum-exp.
+
+    LSE_i = m_i + log(sum_j exp(s_ij - m_i)) with m_i the row maximum (the
+    shift changes nothing mathematically; it keeps exp finite).  Then
+    P = exp(S - LSE).  Returns (P, LSE).
+    """
+    s = _f64(s)
+    m = np.max(s, axis=-1, keepdims=True)
+    lse = m + np.log(np.sum(np.exp(s - m), axis=-1, keepdims=True))
+    p = np.exp(s - lse)
+    return p, lse[..., 0]
+
+
+def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
+                   causal: bool, row_offset: int = 0):
+    """O and LSE for one head: materialise S, then P, then O = P V."""
+    s = attention_scores(q, k, scale, causal, row_offset)
+    p, lse = softmax_with_lse(s)
+    o = p @ _f64(v)
+    return o, lse
+
+
+def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None = None):
+    """Full attention forward for [B, Hq, N, d] queries and [B, Hkv, N, d] K/V.
+
+    Returns (O [B, Hq, N, d] float64, LSE [B, Hq, N] float64).  ``row_chunk``
+    splits each head into blocks of complete query rows (every row still sees
+    its whole key set), which only bounds memory for long sequences.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    o = np.empty((B, Hq, N, v.shape[-1]), dtype=np.float64)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    step = N if row_chunk is None else int(row_chunk)
+    for b in range(B):
+        for h in range(Hq):
+            hk = gqa_kv_head(h, Hq, Hkv)
+            for r0 in range(0, N, step):
+                r1 = min(N, r0 + step)
+                o[b, h, r0:r1], lse[b, h, r0:r1] = attention_head(
+                    q[b, h, r0:r1], k[b, hk], v[b, hk], scale, causal, row_offset=r0)
+    return o, lse
+
+
+def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
+    """O and LSE of selected query rows of head (b, h), each row exact.
+
+    Used for sampled parity checks at sizes where the full oracle is too slow.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    Hq, Hkv = q.shape[1], k.shape[1]
+    hk = gqa_kv_head(h, Hq, Hkv)
+    kk = _f64(k[b, hk])
+    vv = _f64(v[b, hk])
+    out_o = np.empty((rows.size, vv.shape[-1]), dtype=np.float64)
+    out_l = np.empty(rows.size, dtype=np.float64)
+    for i, r in enumerate(rows):
+        qr = _f64(q[b, h, r:r + 1])
+        o_r, l_r = attention_head(qr, kk, vv, scale, causal, row_offset=int(r))
+        out_o[i] = o_r[0]
+        out_l[i] = l_r[0]
+    return out_o, out_l
+
+
+def gather_paged_kv(pool, block_table_row, seq_len: int, page_size: int) -> np.ndarray:
+    """Logical KV rows 0..seq_len-1 of one sequence, read through its block table.
+
+    Token t sits in physical page ``block_table_row[t // page_size]`` at slot
+    ``t % page_size`` ("Paged Attention Kernels": the kernel translates logical
+    positions through the block table).  Returns [seq_len, Hkv, d] in the
+    pool's own dtype (no arithmetic, so the gather is exact).
+    """
+    pool = np.asarray(pool)
+    table = np.asarray(block_table_row)
+    t = np.arange(int(seq_len))
+    pages = table[t // page_size]
+    if seq_len > 0 and (pages.min() < 0 or pages.max() >= pool.shape[0]):
+        raise IndexError("block table entry outside the pool")
+    return pool[pages, t % page_size]
+
+
+def paged_decode(q, k_pool, v_pool, block_table, seq_lens, page_size: int, scale: float):
+    """Single-query decode attention over a paged KV cache.
+
+    q: [S, Hq, d]; pools: [num_pages, page_size, Hkv, d]; block_table:
+    [S, max_pages] int; seq_lens: [S].  The one query of sequence s is its
+    newest token and sees all ``seq_lens[s]`` cached keys (no mask).
+    Returns (O [S, Hq, d] float64, LSE [S, Hq] float64).
+    """
+    q = _f64(q)
+    S, Hq, d = q.shape
+    Hkv = np.asarray(k_pool).shape[2]
+    o = np.empty((S, Hq, d), dtype=np.float64)
+    lse = np.empty((S, Hq), dtype=np.float64)
+    for s in range(S):
+        L = int(seq_lens[s])
+        ks = _f64(gather_paged_kv(k_pool, block_table[s], L, page_size))
+        vs = _f64(gather_paged_kv(v_pool, block_table[s], L, page_size))
+        for h in range(Hq):
+            hk = gqa_kv_head(h, Hq, Hkv)
+            o_h, l_h = attention_head(q[s, h][None, :], ks[:, hk], vs[:, hk], scale, causal=False)
+            o[s, h] = o_h[0]
+            lse[s, h] = l_h[0]
+    return o, lse

@@ -1,0 +1,269 @@
+"""Pins that tie the CPU oracle to facts the pages and the mathematics fix.
+
+Every pin takes an oracle-like module ``o`` (the real ``oracle.attention`` or a
+copy with a planted mistake) and raises ``AssertionError`` when the module
+disagrees with the fact.  None of them re-types the oracle's own vectorised
+formula: they use closed forms, invariants, a scalar brute force written in
+the ratio form sum(w v) / sum(w), PyTorch's fp64 SDPA as a library special
+case, and the pages' printed block-table example.
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _rand(rng, *shape):
+    # bf16-representable values, like the kernels' inputs
+    x = rng.standard_normal(shape).astype(np.float32)
+    return torch.from_numpy(x).to(torch.bfloat16).float().numpy().astype(np.float64)
+
+
+# -- softmax normalisation ---------------------------------------------------
+
+def pin_rows_sum_to_one(o):
+    """Every row of P = softmax(S + M) sums to one (causal and not)."""
+    rng = _rng(11)
+    q, k = _rand(rng, 37, 16), _rand(rng, 37, 16)
+    for causal in (False, True):
+        s = o.attention_scores(q, k, 0.25, causal)
+        p, _ = o.softmax_with_lse(s)
+        assert np.all(np.isfinite(p))
+        assert np.max(np.abs(p.sum(axis=-1) - 1.0)) < 1e-12
+        if causal:
+            assert np.all(p[np.triu_indices(37, 1)] == 0.0)
+
+
+# -- closed forms ------------------------------------------------------------
+
+def pin_constant_v(o):
+    """If every value row equals c, every output row equals c."""
+    rng = _rng(12)
+    B, Hq, Hkv, N, d = 1, 4, 2, 45, 8
+    q = _rand(rng, B, Hq, N, d)
+    k = _rand(rng, B, Hkv, N, d)
+    c = _rand(rng, B, Hkv, 1, d)
+    v = np.broadcast_to(c, (B, Hkv, N, d)).copy()
+    for causal in (False, True):
+        out, _ = o.attention_forward(q, k, v, causal, 0.3)
+        for h in range(Hq):
+            want = c[0, h // (Hq // Hkv), 0]
+            assert np.max(np.abs(out[0, h] - want)) < 1e-12
+
+
+def pin_zero_k(o):
+    """K == 0 makes every visible score 0: O_i is the mean of the visible value
+    rows and LSE_i = log(number of visible keys)."""
+    rng = _rng(13)
+    B, H, N, d = 1, 2, 33, 8
+    q = _rand(rng, B, H, N, d)
+    k = np.zeros((B, H, N, d))
+    v = _rand(rng, B, H, N, d)
+    out, lse = o.attention_forward(q, k, v, True, 0.125)
+    for i in range(N):
+        assert np.max(np.abs(out[0, :, i] - v[0, :, : i + 1].mean(axis=1))) < 1e-12
+        assert np.max(np.abs(lse[0, :, i] - math.log(i + 1))) < 1e-12
+    out, lse = o.attention_forward(q, k, v, False, 0.125)
+    assert np.max(np.abs(out[0] - v[0].mean(axis=1, keepdims=True))) < 1e-12
+    assert np.max(np.abs(lse - math.log(N))) < 1e-12
+
+
+def pin_causal_row0(o):
+    """Causal row 0 sees only key 0: O_0 = v_0 and LSE_0 = scale * q_0 . k_0."""
+    rng = _rng(14)
+    q, k, v = (_rand(rng, 1, 3, 20, 16) for _ in range(3))
+    out, lse = o.attention_forward(q, k, v, True, 0.7)
+    assert np.array_equal(out[0, :, 0], v[0, :, 0])
+    want = 0.7 * np.einsum("hd,hd->h", q[0, :, 0], k[0, :, 0])
+    assert np.max(np.abs(lse[0, :, 0] - want)) < 1e-12
+
+
+def pin_onehot(o):
+    """One key whose score beats all others by ~1000 takes all the weight:
+    exp of the others underflows to exactly 0 in fp64, so O equals that value
+    row exactly and LSE equals that score."""
+    rng = _rng(15)
+    N, d = 24, 8
+    q = np.zeros((1, 1, N, d))
+    q[..., 0] = 1.0
+    k = _rand(rng, 1, 1, N, d) * 0.01
+    v = _rand(rng, 1, 1, N, d)
+    star = 17
+    k[0, 0, star, 0] = 1000.0
+    out, lse = o.attention_forward(q, k, v, False, 1.0)
+    assert np.array_equal(out[0, 0], np.broadcast_to(v[0, 0, star], (N, d)))
+    assert np.max(np.abs(lse[0, 0] - k[0, 0, star, 0])) < 1e-9
+
+
+# -- brute force ---------------------------------------------------------------
+
+def _brute(q, k, v, scale, causal, Hq, Hkv):
+    """Scalar loops, no max shift: O_i = sum_j w_ij v_j / sum_j w_ij with
+    w_ij = exp(scale q_i . k_j), LSE_i = log(sum_j w_ij), sums by math.fsum."""
+    B, _, N, d = q.shape
+    out = np.zeros((B, Hq, N, d))
+    lse = np.zeros((B, Hq, N))
+    g = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // g
+            for i in range(N):
+                ws = []
+                for j in range(N):
+                    if causal and j > i:
+                        continue
+                    dot = math.fsum(float(q[b, h, i, t]) * float(k[b, hk, j, t]) for t in range(d))
+                    ws.append((j, math.exp(scale * dot)))
+                z = math.fsum(w for _, w in ws)
+                lse[b, h, i] = math.log(z)
+                for t in range(d):
+                    out[b, h, i, t] = math.fsum(w * float(v[b, hk, j, t]) for j, w in ws) / z
+    return out, lse
+
+
+def pin_bruteforce(o):
+    """Tiny cases (N <= 8) against the scalar brute force, MHA and GQA."""
+    rng = _rng(16)
+    for (B, Hq, Hkv, N, d, causal, scale) in [
+        (1, 1, 1, 1, 4, True, 0.5),
+        (1, 2, 2, 5, 4, False, 0.5),
+        (2, 4, 2, 7, 3, True, 0.9),
+        (1, 6, 3, 8, 5, False, 0.35),
+        (1, 4, 1, 8, 4, True, 1.3),
+    ]:
+        q = _rand(rng, B, Hq, N, d)
+        k = _rand(rng, B, Hkv, N, d)
+        v = _rand(rng, B, Hkv, N, d)
+        out, lse = o.attention_forward(q, k, v, causal, scale)
+        bo, bl = _brute(q, k, v, scale, causal, Hq, Hkv)
+        assert np.max(np.abs(out - bo)) < 1e-12, (N, causal)
+        assert np.max(np.abs(lse - bl)) < 1e-12, (N, causal)
+
+
+# -- library special case ------------------------------------------------------
+
+def pin_torch_sdpa(o):
+    """PyTorch's CPU fp64 scaled_dot_product_attention (GQA expanded with
+    repeat_interleave) and logsumexp of the masked scores."""
+    rng = _rng(17)
+    for (B, Hq, Hkv, N, d, causal, scale) in [
+        (2, 4, 4, 50, 16, True, 0.25),
+        (1, 8, 2, 67, 32, True, 1 / math.sqrt(32)),
+        (1, 6, 3, 40, 8, False, 0.4),
+    ]:
+        q = _rand(rng, B, Hq, N, d)
+        k = _rand(rng, B, Hkv, N, d)
+        v = _rand(rng, B, Hkv, N, d)
+        out, lse = o.attention_forward(q, k, v, causal, scale)
+        tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+        tk = tk.repeat_interleave(Hq // Hkv, dim=1)
+        tv = tv.repeat_interleave(Hq // Hkv, dim=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale)
+        s = scale * (tq @ tk.transpose(-1, -2))
+        if causal:
+            s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+        ref_lse = torch.logsumexp(s, dim=-1)
+        assert np.max(np.abs(out - ref.numpy())) < 1e-12
+        assert np.max(np.abs(lse - ref_lse.numpy())) < 1e-12
+
+
+# -- paged layout ------------------------------------------------------------------
+
+def pin_block_table_example(o):
+    """The pages' block table: logical blocks 0,1,2,3 live in physical blocks
+    17,4,29,8, and a page holds 16 tokens.  Label every pool slot with its
+    (page, slot) and check where each logical token is read from."""
+    with open(os.path.join(GOLDEN, "block_table_example.json")) as f:
+        ex = json.load(f)
+    ps = ex["page_size"]
+    phys = ex["physical_blocks"]
+    pool = np.zeros((32, ps, 1, 2), dtype=np.int64)
+    for p in range(32):
+        for s in range(ps):
+            pool[p, s, 0] = (p, s)
+    L = len(ex["logical_blocks"]) * ps
+    got = o.gather_paged_kv(pool, np.array(phys), L, ps)
+    for t in range(L):
+        assert tuple(got[t, 0]) == (phys[t // ps], t % ps)
+
+
+def pin_paged_equals_contiguous(o):
+    """Scatter a contiguous KV sequence into randomly chosen pages (shared
+    prefix pages included), read it back through the table: bit-identical.
+    Decode over the pages equals attention of the last query over the
+    contiguous keys."""
+    rng = _rng(18)
+    ps, Hkv, Hq, d = 4, 2, 4, 8
+    lens = [1, 4, 9, 13]
+    num_pages = 16
+    pool_k = _rand(rng, num_pages, ps, Hkv, d)
+    pool_v = _rand(rng, num_pages, ps, Hkv, d)
+    order = rng.permutation(num_pages)
+    table = -np.ones((len(lens), 4), dtype=np.int32)
+    used = 0
+    conts = []
+    for s, L in enumerate(lens):
+        n = -(-L // ps)
+        table[s, :n] = order[used:used + n]
+        used += n
+    table[3, 0] = table[2, 0]  # sequence 3 shares its first page with sequence 2
+    for s, L in enumerate(lens):
+        kc = np.stack([pool_k[table[s, t // ps], t % ps] for t in range(L)])
+        vc = np.stack([pool_v[table[s, t // ps], t % ps] for t in range(L)])
+        assert np.array_equal(o.gather_paged_kv(pool_k, table[s], L, ps), kc)
+        assert np.array_equal(o.gather_paged_kv(pool_v, table[s], L, ps), vc)
+        conts.append((kc, vc))
+    q = _rand(rng, len(lens), Hq, d)
+    out, lse = o.paged_decode(q, pool_k, pool_v, table, np.array(lens), ps, 0.3)
+    for s, (kc, vc) in enumerate(conts):
+        tq = torch.from_numpy(q[s][:, None, :])                       # [Hq,1,d]
+        tk = torch.from_numpy(kc.transpose(1, 0, 2)).repeat_interleave(Hq // Hkv, 0)
+        tv = torch.from_numpy(vc.transpose(1, 0, 2)).repeat_interleave(Hq // Hkv, 0)
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.3)
+        ref_lse = torch.logsumexp(0.3 * (tq @ tk.transpose(-1, -2)), dim=-1)
+        assert np.max(np.abs(out[s] - ref[:, 0].numpy())) < 1e-12
+        assert np.max(np.abs(lse[s] - ref_lse[:, 0].numpy())) < 1e-12
+
+
+def pin_printed_sizes(o):
+    """Numbers the pages print: the N=2048 score matrix holds 4M entries, 16MB
+    in fp32, per head; causal SDPA on (2,16,512,64) returns that shape."""
+    with open(os.path.join(GOLDEN, "printed_values.json")) as f:
+        pv = json.load(f)
+    sm = pv["score_matrix"]
+    N = sm["N"]
+    q = np.ones((N, 1))
+    s = o.attention_scores(q, q, 1.0, False)
+    assert s.size == sm["elements"]
+    assert s.astype(np.float32).nbytes == sm["bytes_fp32"]
+    shp = pv["sdpa_example"]["shape"]
+    small = [1, 2, 24, shp[3]]  # same head dim; fewer heads/rows keeps it fast
+    rng = _rng(19)
+    q, k, v = (_rand(rng, *small) for _ in range(3))
+    out, lse = o.attention_forward(q, k, v, pv["sdpa_example"]["causal"], 0.125)
+    assert list(out.shape) == small and list(lse.shape) == small[:3]
+
+
+ALL_PINS = [
+    pin_rows_sum_to_one,
+    pin_constant_v,
+    pin_zero_k,
+    pin_causal_row0,
+    pin_onehot,
+    pin_bruteforce,
+    pin_torch_sdpa,
+    pin_block_table_example,
+    pin_paged_equals_contiguous,
+    pin_printed_sizes,
+]

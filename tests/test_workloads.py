@@ -1,0 +1,93 @@
+"""Seeded input generators: determinism, shapes, block-table structure (CPU)."""
+
+import math
+
+import torch
+
+from attention_flashattention_fwd_04_b200 import workloads as W
+
+
+def test_prefill_inputs_are_seeded_and_shaped():
+    cfg = W.PREFILL_CONFIGS["tiny"]
+    a = W.make_prefill_inputs(cfg)
+    b = W.make_prefill_inputs(cfg)
+    for x, y in zip(a, b):
+        assert x.dtype == torch.bfloat16 and x.is_contiguous()
+        assert torch.equal(x, y)
+    assert a[0].shape == (1, 2, 128, 64)
+    assert a[1].shape == (1, 2, 128, 64)
+
+
+def test_scale_is_fp32_rounded_inverse_sqrt():
+    for cfg in W.PREFILL_CONFIGS.values():
+        s = cfg.scale
+        assert s == float(torch.tensor(1 / math.sqrt(cfg.d), dtype=torch.float32))
+    assert W.PREFILL_CONFIGS["tiny"].scale == 0.125
+
+
+def test_gqa_config_shapes_and_value_scale():
+    cfg = W.PrefillConfig("t", 1, 8, 2, 256, 128, True, 3, value_scale=0.5)
+    q, k, v = W.make_prefill_inputs(cfg)
+    assert q.shape == (1, 8, 256, 128) and k.shape == (1, 2, 256, 128)
+    assert 0.4 < q.float().std().item() < 0.6
+
+
+def test_k_offset_is_per_position_and_shared_across_heads():
+    cfg = W.PrefillConfig("t", 1, 2, 2, 512, 128, True, 5, k_offset_sigma=2.0)
+    q, k, v = W.make_prefill_inputs(cfg)
+    row_means = k.float().mean(dim=-1)  # [1, 2, N]
+    # the offset dominates the row mean and is the same for both heads
+    assert torch.corrcoef(torch.stack([row_means[0, 0], row_means[0, 1]]))[0, 1] > 0.95
+    assert 1.5 < row_means[0, 0].std().item() < 2.5
+
+
+def test_decode_block_table_is_a_permutation_with_padding():
+    cfg = W.DecodeConfig("t", 7, 8, 2, 64, 16, 1, 300, 9)
+    inp = W.make_decode_inputs(cfg)
+    L = inp["seq_lens"].long()
+    table = inp["block_table"]
+    ps = inp["page_size"]
+    pages = (L + ps - 1) // ps
+    assert int(pages.sum()) == inp["num_pages"]
+    assert inp["k_pool"].shape == (inp["num_pages"], ps, 2, 64)
+    ids = []
+    for s in range(cfg.num_seqs):
+        n = int(pages[s])
+        ids += table[s, :n].tolist()
+        assert bool((table[s, n:] == -1).all())
+    assert sorted(ids) == list(range(inp["num_pages"]))
+    assert int(L.min()) >= 1 and int(L.max()) <= 300
+    again = W.make_decode_inputs(cfg)
+    assert torch.equal(again["block_table"], table)
+    assert torch.equal(again["k_pool"], inp["k_pool"])
+
+
+def test_decode_poison_fills_only_unused_tail_slots():
+    cfg = W.DecodeConfig("t", 4, 4, 2, 32, 16, 1, 100, 10)
+    inp = W.make_decode_inputs(cfg, poison_tail=True, seq_lens=[1, 16, 17, 33])
+    kp = inp["k_pool"].float()
+    table = inp["block_table"]
+    for s, L in enumerate([1, 16, 17, 33]):
+        n = -(-L // 16)
+        for p in range(n):
+            page = kp[int(table[s, p])]
+            for slot in range(16):
+                t = p * 16 + slot
+                assert bool(torch.isnan(page[slot]).all()) == (t >= L)
+
+
+def test_paged_decode_default_config_sizes():
+    cfg = W.DECODE_CONFIGS["paged_decode"]
+    assert cfg.table_width == 512
+    g = torch.Generator().manual_seed(cfg.seed)
+    L = torch.randint(cfg.min_len, cfg.max_len + 1, (cfg.num_seqs,), generator=g)
+    assert 512 <= int(L.min()) and int(L.max()) <= 8192
+    b = W.decode_kv_bytes(L, cfg.Hkv, cfg.d, cfg.Hq)
+    assert b > float(L.sum()) * 4096
+
+
+def test_flop_convention():
+    c2 = W.PREFILL_CONFIGS["causal_mha"]
+    assert abs(W.prefill_flops(c2) - 68.72e9) / 68.72e9 < 1e-3
+    c3 = W.PREFILL_CONFIGS["causal_gqa"]
+    assert abs(W.prefill_flops(c3) - 549.76e9) / 549.76e9 < 1e-3
