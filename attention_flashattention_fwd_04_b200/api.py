@@ -1,0 +1,195 @@
+"""ctypes binding over the C ABI in ``include/attn_b200.h``.
+
+Argument marshalling only: every step of the attention runs in the CUDA
+kernels of ``libattn_b200.so``.  PyTorch supplies device memory (outputs,
+workspace) and the current stream.  There is no CPU or PyTorch fallback: if
+the library is missing or a call fails, this module raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+from .build import INCLUDE, LIB_PATH
+
+ATTN_OK = 0
+_STATUS_NAMES = {
+    0: "ATTN_OK",
+    1: "ATTN_ERR_NULL",
+    2: "ATTN_ERR_SHAPE",
+    3: "ATTN_ERR_ALIGN",
+    4: "ATTN_ERR_WORKSPACE",
+    5: "ATTN_ERR_UNSUPPORTED",
+    6: "ATTN_ERR_LAUNCH",
+    7: "ATTN_ERR_DEVICE",
+}
+
+_c_p = ctypes.c_void_p
+_c_i = ctypes.c_int
+_c_f = ctypes.c_float
+_c_sz = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/attn_b200.h
+SIGNATURES = {
+    "attn_abi_version": (_c_i, []),
+    "attn_status_string": (ctypes.c_char_p, [_c_i]),
+    "attn_last_cuda_error": (_c_i, []),
+    "attn_fwd": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p]),
+    "paged_attn_decode_split_tokens": (_c_i, [_c_i, _c_i, _c_i, _c_i]),
+    "paged_attn_decode_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
+    "paged_attn_decode": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i,
+                                 _c_i, _c_i, _c_f, _c_p, _c_sz, _c_p]),
+    "attn_device_status": (_c_i, [_c_p, ctypes.POINTER(ctypes.c_uint)]),
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        name = _STATUS_NAMES.get(status, str(status))
+        msg = f"{what}: {name} ({status_string(status)})"
+        if status == 6:
+            msg += f"; cudaError {lib().attn_last_cuda_error()}"
+        super().__init__(msg)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library (loaded on first use)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m attention_flashattention_fwd_04_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/attn_b200.h."""
+    with open(os.path.join(INCLUDE, "attn_b200.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(\w+)\s*\(", text, flags=re.M)
+
+
+def status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != ATTN_OK:
+        raise AttnError(rc, what)
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _require(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
+             scale: float | None = None, out: torch.Tensor | None = None,
+             lse: torch.Tensor | None = None, stream=None):
+    """Fused attention forward.  q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 CUDA.
+
+    Returns (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32).
+    """
+    _require(q, "q", torch.bfloat16, 4)
+    _require(k, "k", torch.bfloat16, 4)
+    _require(v, "v", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} do not match q {tuple(q.shape)}")
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _require(out, "out", torch.bfloat16, 4)
+    _require(lse, "lse", torch.float32, 3)
+    rc = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                        B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
+    _check(rc, "attn_fwd")
+    return out, lse
+
+
+def paged_attn_decode_split_tokens(num_seqs: int, Hkv: int, max_pages: int, page_size: int) -> int:
+    return int(lib().paged_attn_decode_split_tokens(num_seqs, Hkv, max_pages, page_size))
+
+
+def paged_attn_decode_workspace_bytes(num_seqs: int, Hq: int, d: int, max_pages: int, page_size: int) -> int:
+    return int(lib().paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_pages, page_size))
+
+
+def paged_attn_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                      block_table: torch.Tensor, seq_lens: torch.Tensor, scale: float | None = None,
+                      workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                      lse: torch.Tensor | None = None, stream=None):
+    """Decode attention over a paged KV cache.
+
+    q [S,Hq,d] bf16; k_pool/v_pool [num_pages,page_size,Hkv,d] bf16;
+    block_table [S,max_pages] int32; seq_lens [S] int32 (all on the GPU).
+    Returns (o [S,Hq,d] bf16, lse [S,Hq] fp32).
+    """
+    _require(q, "q", torch.bfloat16, 3)
+    _require(k_pool, "k_pool", torch.bfloat16, 4)
+    _require(v_pool, "v_pool", torch.bfloat16, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(seq_lens, "seq_lens", torch.int32, 1)
+    S, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_pool.shape
+    if dk != d or v_pool.shape != k_pool.shape:
+        raise ValueError("pool shapes do not match q")
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table / seq_lens do not match the number of sequences")
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    need = paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, page_size)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    rc = lib().paged_attn_decode(
+        q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+        page_size, out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages, float(scale),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    _check(rc, "paged_attn_decode")
+    return out, lse
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device error bits."""
+    bits = ctypes.c_uint(0)
+    rc = lib().attn_device_status(_stream_handle(stream), ctypes.byref(bits))
+    if rc not in (ATTN_OK, 7):
+        raise AttnError(rc, "attn_device_status")
+    return int(bits.value)

@@ -1,0 +1,290 @@
+// Host side of the C ABI declared in include/attn_b200.h: argument checks,
+// TMA tensor-map encoding, split planning and kernel launches.  Nothing here
+// allocates device memory or synchronises (except attn_device_status, whose
+// job is to synchronise).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn_b200.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+int fail_cuda(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return ATTN_ERR_LAUNCH;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres{};
+    const cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                                           cudaEnableDefault, &qres);
+    if (e == cudaSuccess && qres == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
+// dims[0] is the contiguous dimension; strides are the byte strides of
+// dims[1] and dims[2].
+bool encode_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1, stride2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool misaligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPrefillStages = 2;
+
+template <int D, bool CAUSAL>
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const attn::PrefillParams& p, cudaStream_t stream) {
+  using L = attn::PrefillLayout<D, kPrefillStages>;
+  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, kPrefillStages>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return fail_cuda(e);
+  const unsigned grid = static_cast<unsigned>(p.num_q_tiles) * static_cast<unsigned>(p.B * p.Hq);
+  kernel<<<grid, attn::kPrefillThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail_cuda(e);
+  return ATTN_OK;
+}
+
+int decode_heads_per_cta(int Hkv) {
+  int hb = 1;
+  while (hb < 8 && Hkv % (hb * 2) == 0) hb *= 2;
+  return hb;
+}
+
+int split_tokens_for(int num_seqs, int Hkv, int max_pages, int page_size) {
+  (void)num_seqs;
+  (void)Hkv;
+  (void)max_pages;
+  (void)page_size;
+  return 256;
+}
+
+struct DecodePlan {
+  int split_tokens = 0;
+  int max_splits = 0;
+  size_t o_bytes = 0;
+  size_t lse_offset = 0;
+  size_t total = 0;
+};
+
+bool decode_plan(int num_seqs, int Hq, int Hkv, int d, int max_pages, int page_size, DecodePlan* out) {
+  if (num_seqs < 1 || Hq < 1 || max_pages < 1 || page_size < 1 || (d != 64 && d != 128)) return false;
+  const long long max_tokens = static_cast<long long>(max_pages) * page_size;
+  if (max_tokens > INT_MAX) return false;
+  DecodePlan pl;
+  pl.split_tokens = split_tokens_for(num_seqs, Hkv, max_pages, page_size);
+  pl.max_splits = static_cast<int>((max_tokens + pl.split_tokens - 1) / pl.split_tokens);
+  const size_t rows = static_cast<size_t>(num_seqs) * Hq * pl.max_splits;
+  pl.o_bytes = rows * d * sizeof(float);
+  pl.lse_offset = (pl.o_bytes + 255) & ~static_cast<size_t>(255);
+  pl.total = pl.lse_offset + rows * sizeof(float);
+  *out = pl;
+  return true;
+}
+
+template <int D, int HB>
+int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const attn::DecodeParams& p,
+                  attn_bf16* o, float* lse, cudaStream_t stream) {
+  using L = attn::DecodeLayout<D, HB>;
+  auto split_kernel = attn::decode_split_kernel<D, HB>;
+  cudaError_t e = cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return fail_cuda(e);
+  const dim3 grid(static_cast<unsigned>(p.max_splits), static_cast<unsigned>(p.S),
+                  static_cast<unsigned>(p.Hkv / HB));
+  split_kernel<<<grid, 32 * (HB + 1), L::kAlloc, stream>>>(tk, tv, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail_cuda(e);
+  const long long warps = static_cast<long long>(p.S) * p.Hq;
+  const unsigned mgrid = static_cast<unsigned>((warps * 32 + 255) / 256);
+  attn::decode_merge_kernel<D><<<mgrid, 256, 0, stream>>>(p, reinterpret_cast<__nv_bfloat16*>(o), lse);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return fail_cuda(e);
+  return ATTN_OK;
+}
+
+template <int D>
+int dispatch_decode_hb(int hb, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const attn::DecodeParams& p, attn_bf16* o, float* lse, cudaStream_t stream) {
+  switch (hb) {
+    case 8: return launch_decode<D, 8>(tk, tv, p, o, lse, stream);
+    case 4: return launch_decode<D, 4>(tk, tv, p, o, lse, stream);
+    case 2: return launch_decode<D, 2>(tk, tv, p, o, lse, stream);
+    default: return launch_decode<D, 1>(tk, tv, p, o, lse, stream);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return 1; }
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_NULL: return "a required pointer is NULL";
+    case ATTN_ERR_SHAPE: return "a size is out of range or inconsistent";
+    case ATTN_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case ATTN_ERR_UNSUPPORTED: return "input valid but not supported by this build";
+    case ATTN_ERR_LAUNCH: return "CUDA refused the launch";
+    case ATTN_ERR_DEVICE: return "a kernel recorded a runtime error";
+    default: return "unknown status";
+  }
+}
+
+int attn_last_cuda_error(void) { return t_last_cuda_error; }
+
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
+             int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_SHAPE;
+  if (d != 64 && d != 128) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return ATTN_ERR_SHAPE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_SHAPE;
+  const long long bh = static_cast<long long>(B) * Hq;
+  const long long tiles = (static_cast<long long>(N) + 127) / 128;
+  if (bh > INT_MAX || tiles * bh > INT_MAX) return ATTN_ERR_SHAPE;
+  if (misaligned16(q) || misaligned16(k) || misaligned16(v) || misaligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return ATTN_ERR_ALIGN;
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t row_bytes = static_cast<uint64_t>(d) * 2;
+  const uint64_t head_bytes = row_bytes * static_cast<uint64_t>(N);
+  if (!encode_3d(&tq, q, d, N, static_cast<uint64_t>(B) * Hq, row_bytes, head_bytes, 64, 128, 1) ||
+      !encode_3d(&tk, k, d, N, static_cast<uint64_t>(B) * Hkv, row_bytes, head_bytes, 64, 128, 1) ||
+      !encode_3d(&tv, v, d, N, static_cast<uint64_t>(B) * Hkv, row_bytes, head_bytes, 64, 128, 1))
+    return fail_cuda(cudaErrorInvalidValue);
+
+  attn::PrefillParams p;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.num_q_tiles = static_cast<int>(tiles);
+  p.scale_log2 = scale * kLog2e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch_prefill<128, true>(tq, tk, tv, p, s) : launch_prefill<128, false>(tq, tk, tv, p, s);
+  return causal ? launch_prefill<64, true>(tq, tk, tv, p, s) : launch_prefill<64, false>(tq, tk, tv, p, s);
+}
+
+int paged_attn_decode_split_tokens(int num_seqs, int Hkv, int max_pages, int page_size) {
+  return split_tokens_for(num_seqs, Hkv, max_pages, page_size);
+}
+
+size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_pages, int page_size) {
+  DecodePlan pl;
+  if (!decode_plan(num_seqs, Hq, 1, d, max_pages, page_size, &pl)) return 0;
+  return pl.total;
+}
+
+int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                      const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                      attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
+                      int max_pages, int num_pages, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !o || !lse) return ATTN_ERR_NULL;
+  if (num_seqs < 1 || Hq < 1 || Hkv < 1 || max_pages < 1 || num_pages < 1 || page_size < 1)
+    return ATTN_ERR_SHAPE;
+  if (d != 64 && d != 128) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_SHAPE;
+  if (num_seqs > 65535 || Hkv > 65535) return ATTN_ERR_SHAPE;
+  if (static_cast<long long>(num_pages) * page_size > INT_MAX) return ATTN_ERR_SHAPE;
+  if (page_size % 16 != 0 || page_size > 256) return ATTN_ERR_UNSUPPORTED;
+  if (Hq / Hkv > 16) return ATTN_ERR_UNSUPPORTED;
+  DecodePlan pl;
+  if (!decode_plan(num_seqs, Hq, Hkv, d, max_pages, page_size, &pl)) return ATTN_ERR_SHAPE;
+  if (!workspace) return ATTN_ERR_WORKSPACE;
+  if (workspace_bytes < pl.total) return ATTN_ERR_WORKSPACE;
+  if (misaligned16(q) || misaligned16(k_pool) || misaligned16(v_pool) || misaligned16(o) ||
+      misaligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0)
+    return ATTN_ERR_ALIGN;
+
+  const int hb = decode_heads_per_cta(Hkv);
+  CUtensorMap tk, tv;
+  const uint64_t token_bytes = static_cast<uint64_t>(Hkv) * d * 2;
+  const uint64_t head_bytes = static_cast<uint64_t>(d) * 2;
+  const uint64_t rows = static_cast<uint64_t>(num_pages) * page_size;
+  if (!encode_3d(&tk, k_pool, d, rows, Hkv, token_bytes, head_bytes, 64, attn::kDecodeChunk, hb) ||
+      !encode_3d(&tv, v_pool, d, rows, Hkv, token_bytes, head_bytes, 64, attn::kDecodeChunk, hb))
+    return fail_cuda(cudaErrorInvalidValue);
+
+  attn::DecodeParams p;
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.lse_offset);
+  p.S = num_seqs;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.page_size = page_size;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.max_splits = pl.max_splits;
+  p.split_tokens = pl.split_tokens;
+  p.scale_log2 = scale * kLog2e;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128) return dispatch_decode_hb<128>(hb, tk, tv, p, o, lse, s);
+  return dispatch_decode_hb<64>(hb, tk, tv, p, o, lse, s);
+}
+
+int attn_device_status(void* stream, unsigned int* bits) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  unsigned int word = 0;
+  e = cudaMemcpyFromSymbol(&word, attn::g_attn_device_error, sizeof(word));
+  if (e != cudaSuccess) return fail_cuda(e);
+  if (bits) *bits = word;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(attn::g_attn_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail_cuda(e);
+    return ATTN_ERR_DEVICE;
+  }
+  return ATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,594 @@
+#!/usr/bin/env python
+"""Throughput of the attention hot path on B200, as a fraction of peak.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the causal prefill of B=4, H=16, N=2048, d=128 (fused QK^T, mask, online
+softmax, PV, LSE) followed by the paged-KV decode of 64 sequences (Hq=32,
+Hkv=8, d=128, 16-token pages, lengths 512..8192): split-KV pass + merge.
+
+value = (prefill FLOPs / peak bf16 FLOP/s + decode bytes / peak HBM B/s)
+        summed over ranks / max-over-ranks step time,
+i.e. the time-weighted fraction of the measured B200 peaks the step reaches
+(per GPU it is at most ~1; over N GPUs it adds up, weak scaling).  The
+separate prefill TFLOP/s and decode GB/s are in the line too.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       [--workload default|causal_mha|causal_gqa|long_causal|paged_decode]
+Under torchrun each rank runs its own batch (seed offset by rank), no
+collective on the data path; rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from attention_flashattention_fwd_04_b200 import workloads as W  # noqa: E402
+
+METRIC = "causal prefill TFLOP/s and paged-decode KV GB/s, as fraction of B200 peaks"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+KERNEL_SOURCES = ["attn_api.cu", "prefill_sm100.cuh", "decode_sm100.cuh", "ptx.cuh", "tmem_ldst.cuh"]
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"])
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "attention_flashattention_fwd_04_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    out = {}
+    try:
+        with open(path) as f:
+            for line in f:
+                line = line.strip()
+                if not line or line.startswith("#"):
+                    continue
+                kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
+                if "kernel" in kv and "dram_bytes_per_launch" in kv:
+                    out[kv["kernel"]] = (kv.get("sha"), float(kv["dram_bytes_per_launch"]))
+    except OSError:
+        return {}
+    sha = kernel_source_hash()
+    return {k: v for k, (s, v) in out.items() if s == sha}
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own independent batch (weak scaling)."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device, period_s: float = 0.01):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            try:  # NVML numbers GPUs physically; match the CUDA device by UUID
+                uuid = str(torch.cuda.get_device_properties(device).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch.device(device).index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: report no samples
+            self._nvml = None
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                bits = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+class Step:
+    """Device-resident inputs/outputs for one rank and the calls of one step."""
+
+    def __init__(self, workload: str, rank: int, device):
+        from attention_flashattention_fwd_04_b200 import api
+        self.api = api
+        self.device = device
+        self.prefill_cfg = None
+        self.decode_cfg = None
+        if workload in ("default", "causal_mha", "causal_gqa", "long_causal", "tiny"):
+            name = "causal_mha" if workload == "default" else workload
+            base = W.PREFILL_CONFIGS[name]
+            self.prefill_cfg = W.PrefillConfig(base.name, base.B, base.Hq, base.Hkv, base.N, base.d, base.causal,
+                                               shard_seed(base.seed, rank), base.value_scale, base.k_offset_sigma)
+        if workload in ("default", "paged_decode"):
+            base = W.DECODE_CONFIGS["paged_decode"]
+            self.decode_cfg = W.DecodeConfig(base.name, base.num_seqs, base.Hq, base.Hkv, base.d, base.page_size,
+                                             base.min_len, base.max_len, shard_seed(base.seed, rank))
+        self.host = {}
+        self.dev = {}
+        self.flops = 0.0
+        self.bytes = 0.0
+        if self.prefill_cfg is not None:
+            c = self.prefill_cfg
+            q, k, v = W.make_prefill_inputs(c)
+            self.host.update(q=q, k=k, v=v)
+            self.flops = W.prefill_flops(c)
+        if self.decode_cfg is not None:
+            c = self.decode_cfg
+            inp = W.make_decode_inputs(c)
+            self.decode_inp = inp
+            self.host.update(dq=inp["q"], k_pool=inp["k_pool"], v_pool=inp["v_pool"],
+                             block_table=inp["block_table"], seq_lens=inp["seq_lens"])
+            self.bytes = W.decode_kv_bytes(inp["seq_lens"], c.Hkv, c.d, c.Hq, c.page_size)
+        for name, t in self.host.items():
+            self.dev[name] = t.to(device)
+        self._alloc_outputs()
+
+    def _alloc_outputs(self):
+        api, dev = self.api, self.device
+        if self.prefill_cfg is not None:
+            q = self.dev["q"]
+            self.dev["o"] = torch.empty_like(q)
+            self.dev["lse"] = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        if self.decode_cfg is not None:
+            c, inp = self.decode_cfg, self.decode_inp
+            need = api.paged_attn_decode_workspace_bytes(c.num_seqs, c.Hq, c.d, inp["max_pages"], c.page_size)
+            self.dev["ws"] = torch.empty(need, dtype=torch.uint8, device=dev)
+            self.dev["do"] = torch.empty_like(self.dev["dq"])
+            self.dev["dlse"] = torch.empty((c.num_seqs, c.Hq), dtype=torch.float32, device=dev)
+
+    def launches_per_step(self) -> int:
+        return (1 if self.prefill_cfg is not None else 0) + (2 if self.decode_cfg is not None else 0)
+
+    def run_prefill(self, d=None):
+        d = d or self.dev
+        c = self.prefill_cfg
+        self.api.attn_fwd(d["q"], d["k"], d["v"], c.causal, c.scale, out=d["o"], lse=d["lse"])
+
+    def run_decode(self, d=None):
+        d = d or self.dev
+        c = self.decode_cfg
+        self.api.paged_attn_decode(d["dq"], d["k_pool"], d["v_pool"], d["block_table"], d["seq_lens"], c.scale,
+                                   workspace=self.dev["ws"], out=d["do"], lse=d["dlse"])
+
+    def ideal_seconds(self, peaks) -> float:
+        return self.flops / (peaks["bf16_tflops"] * 1e12) + self.bytes / (peaks["hbm_gbs"] * 1e9)
+
+
+def config_dict(step: Step, n_gpus: int):
+    cfg = {"workload": None, "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single"}
+    parts = []
+    if step.prefill_cfg is not None:
+        c = step.prefill_cfg
+        parts.append(f"causal prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}")
+        cfg["prefill"] = {"B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "N": c.N, "d": c.d, "causal": c.causal,
+                          "scale": c.scale, "seed": c.seed, "value_scale": c.value_scale,
+                          "k_offset_sigma": c.k_offset_sigma, "flops": step.flops}
+    if step.decode_cfg is not None:
+        c = step.decode_cfg
+        L = step.decode_inp["seq_lens"]
+        parts.append(f"paged decode {c.num_seqs} seqs Hq={c.Hq} Hkv={c.Hkv} d={c.d} page={c.page_size}")
+        cfg["decode"] = {"num_seqs": c.num_seqs, "Hq": c.Hq, "Hkv": c.Hkv, "d": c.d, "page_size": c.page_size,
+                         "len_range": [c.min_len, c.max_len], "total_tokens": int(L.sum()),
+                         "num_pages": step.decode_inp["num_pages"], "seed": c.seed, "bytes": step.bytes}
+    cfg["workload"] = " + ".join(parts)
+    if step.decode_cfg is not None:
+        cfg["l2"] = "inputs larger than L2: the decode pass streams >1 GB of KV through the 126 MB L2 every step"
+    else:
+        cfg["l2"] = "L2 flushed between steps (256 MB write)"
+    return cfg
+
+
+# ----------------------------------------------------------------------------- CPU oracle legs
+
+def oracle_sample(step_cfgs, budget_s: float, per_call=False):
+    """Times the CPU oracle (as it stands) on a bounded sample of the workload.
+
+    Returns (work dict, seconds, sample description).  The sample walks the
+    prefill heads (complete heads, every row) and the decode sequences in
+    order until `budget_s` of CPU time has been used.
+    """
+    import numpy as np
+
+    import oracle
+
+    prefill_cfg, decode_cfg, host, decode_inp = step_cfgs
+    flops = 0.0
+    nbytes = 0.0
+    done_heads = 0
+    done_seqs = 0
+    t0 = time.perf_counter()
+    if prefill_cfg is not None:
+        c = prefill_cfg
+        q, k, v = (host[n].float().numpy() for n in ("q", "k", "v"))
+        rows = c.N if not per_call else 128
+        for b in range(c.B):
+            for h in range(c.Hq):
+                hk = h * c.Hkv // c.Hq
+                r0 = c.N - rows
+                oracle.attention_head(q[b, h, r0:], k[b, hk], v[b, hk], c.scale, c.causal, row_offset=r0)
+                # causal work of rows r0..N-1: sum over rows of (row+1) keys
+                keys = (rows * (r0 + 1 + c.N)) / 2.0 if c.causal else rows * c.N
+                flops += 4.0 * keys * c.d
+                done_heads += 1
+                if time.perf_counter() - t0 > budget_s / (2 if decode_cfg is not None else 1):
+                    break
+            else:
+                continue
+            break
+    t1 = time.perf_counter()
+    if decode_cfg is not None:
+        c = decode_cfg
+        kp = host["k_pool"].float().numpy()
+        vp = host["v_pool"].float().numpy()
+        qd = host["dq"].float().numpy().astype(np.float64)
+        table = host["block_table"].numpy()
+        lens = host["seq_lens"].numpy()
+        for s in range(c.num_seqs):
+            oracle.paged_decode(qd[s:s + 1], kp, vp, table[s:s + 1], lens[s:s + 1], c.page_size, c.scale)
+            nbytes += float(lens[s]) * 2 * c.Hkv * c.d * 2
+            done_seqs += 1
+            if time.perf_counter() - t1 > budget_s / (2 if prefill_cfg is not None else 1) or per_call:
+                break
+    seconds = time.perf_counter() - t0
+    desc = []
+    if prefill_cfg is not None:
+        desc.append(f"{done_heads} prefill heads ({'last 128 rows' if per_call else 'all rows'})")
+    if decode_cfg is not None:
+        desc.append(f"{done_seqs} decode sequences")
+    return {"flops": flops, "bytes": nbytes}, seconds, ", ".join(desc)
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle as it stands, on bounded samples."""
+    if rank != 0:
+        return None
+    peaks = load_peaks()
+    step = StepHost(args.workload)
+    cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp)
+    for _ in range(args.warmup):
+        oracle_sample(cfgs, 0.0, per_call=True)
+    work_f = work_b = secs = 0.0
+    desc = ""
+    for _ in range(args.steps):
+        w, s, desc = oracle_sample(cfgs, 0.0, per_call=True)
+        work_f += w["flops"]
+        work_b += w["bytes"]
+        secs += s
+    ideal = work_f / (peaks["bf16_tflops"] * 1e12) + work_b / (peaks["hbm_gbs"] * 1e9)
+    value = ideal / secs
+    line = {
+        "metric": METRIC, "value": value, "unit": unit_string(), "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "config": step.config,
+        "cpu_baseline": {"value": value, "unit": unit_string(), "cores": cpu_threads(), "kind": "oracle",
+                         "sample": f"per step: {desc}"},
+        "e2e": {"value": value, "unit": unit_string(), "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+class StepHost:
+    """Host-only inputs for the reference arm (no GPU needed)."""
+
+    def __init__(self, workload):
+        self.prefill_cfg = self.decode_cfg = None
+        self.host = {}
+        self.decode_inp = None
+        parts = []
+        if workload in ("default", "causal_mha", "causal_gqa", "long_causal", "tiny"):
+            name = "causal_mha" if workload == "default" else workload
+            self.prefill_cfg = W.PREFILL_CONFIGS[name]
+            q, k, v = W.make_prefill_inputs(self.prefill_cfg)
+            self.host.update(q=q, k=k, v=v)
+            c = self.prefill_cfg
+            parts.append(f"causal prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}")
+        if workload in ("default", "paged_decode"):
+            self.decode_cfg = W.DECODE_CONFIGS["paged_decode"]
+            inp = W.make_decode_inputs(self.decode_cfg)
+            self.decode_inp = inp
+            self.host.update(dq=inp["q"], k_pool=inp["k_pool"], v_pool=inp["v_pool"],
+                             block_table=inp["block_table"], seq_lens=inp["seq_lens"])
+            c = self.decode_cfg
+            parts.append(f"paged decode {c.num_seqs} seqs Hq={c.Hq} Hkv={c.Hkv} d={c.d} page={c.page_size}")
+        self.config = {"workload": " + ".join(parts), "parallelism": "single"}
+
+
+def unit_string() -> str:
+    return "fraction of B200 peak (time-weighted: prefill bf16 FLOP/s, decode HBM B/s), summed over GPUs"
+
+
+def run_ours(args, world, rank, local_rank):
+    from attention_flashattention_fwd_04_b200 import api
+    from attention_flashattention_fwd_04_b200.build import build
+
+    build()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    peaks = load_peaks()
+    step = Step(args.workload, rank, device)
+    stream = torch.cuda.current_stream()
+    flush = None
+    if step.decode_cfg is None:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+
+    def one_step(ev=None):
+        if step.prefill_cfg is not None:
+            if ev is not None:
+                ev[0].record(stream)
+            step.run_prefill()
+            if ev is not None:
+                ev[1].record(stream)
+        if step.decode_cfg is not None:
+            step.run_decode()
+            if ev is not None:
+                ev[2].record(stream)
+        if flush is not None:
+            flush.fill_(1)
+
+    for _ in range(args.warmup):
+        one_step()
+    if api.device_status() != 0:
+        raise RuntimeError("a kernel reported a device error during warm-up")
+
+    # ---- device-resident timing
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device) as clocks:
+        start.record(stream)
+        for i in range(args.steps):
+            one_step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    if api.device_status() != 0:
+        raise RuntimeError("a kernel reported a device error in the timed region")
+    total_s = start.elapsed_time(end) / 1e3
+    t_prefill = t_decode = 0.0
+    for i in range(args.steps):
+        if step.prefill_cfg is not None:
+            t_prefill += evs[i][0].elapsed_time(evs[i][1]) / 1e3
+        if step.decode_cfg is not None:
+            a = evs[i][1] if step.prefill_cfg is not None else (evs[i - 1][2] if i > 0 else start)
+            t_decode += a.elapsed_time(evs[i][2]) / 1e3
+    t_max = max_over_ranks(total_s, world, device)
+    ideal_sum = sum_over_ranks(step.ideal_seconds(peaks) * args.steps, world, device)
+    value = ideal_sum / t_max
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = run_e2e(step, args, world, device, peaks)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": unit_string(), "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * t_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(step, world),
+        "gpu_launches": step.launches_per_step() * args.steps,
+        "clocks": clocks.summary(),
+        "peaks": peaks,
+    }
+    kernels = {}
+    if step.prefill_cfg is not None:
+        per = t_prefill / args.steps
+        tfl = step.flops / per / 1e12
+        kernels["prefill_fwd_kernel"] = {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"],
+                                         "unit": "TFLOP/s", "frac": tfl / peaks["bf16_tflops"],
+                                         "us_per_launch": per * 1e6, "algorithmic": step.flops}
+        line["prefill_tflops"] = tfl
+    if step.decode_cfg is not None:
+        per = t_decode / args.steps
+        gbs = step.bytes / per / 1e9
+        kernels["decode (split + merge)"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                                             "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                                             "us_per_launch": per * 1e6, "algorithmic": step.bytes}
+        line["decode_kv_gbs"] = gbs
+    dominant = max(kernels, key=lambda k: kernels[k]["us_per_launch"])
+    traffic = load_traffic()
+    dk = kernels[dominant]
+    tkey = "prefill_fwd_kernel" if dominant.startswith("prefill") else "decode_split_kernel"
+    line["roofline"] = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
+                        "unit": dk["unit"], "frac": dk["frac"], "traffic": traffic.get(tkey),
+                        "peak_source": f"{peaks['source']} (burst)"}
+    line["kernels"] = kernels
+    line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        w, secs, desc = oracle_sample((step.prefill_cfg, step.decode_cfg, step.host,
+                                       getattr(step, "decode_inp", None)), args.cpu_seconds)
+        ideal = w["flops"] / (peaks["bf16_tflops"] * 1e12) + w["bytes"] / (peaks["hbm_gbs"] * 1e9)
+        cpu = {"value": ideal / secs, "unit": unit_string(), "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{desc}; {secs:.1f} s"}
+        if w["flops"]:
+            cpu["prefill_gflops"] = w["flops"] / secs / 1e9
+        if w["bytes"]:
+            cpu["decode_gbs"] = w["bytes"] / secs / 1e9
+        line["cpu_baseline"] = cpu
+    return line
+
+
+def run_e2e(step: Step, args, world, device, peaks):
+    """Same metric through the public API, host buffers: every step copies its
+    inputs from pinned host memory and reads the results back."""
+    pinned = {n: t.pin_memory() for n, t in step.host.items()}
+    outs = {}
+    for n in ("o", "lse", "do", "dlse"):
+        if n in step.dev:
+            outs[n] = torch.empty(step.dev[n].shape, dtype=step.dev[n].dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    steps = max(1, min(args.steps, args.e2e_steps))
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for n, t in pinned.items():
+            step.dev[n].copy_(t, non_blocking=True)
+        if step.prefill_cfg is not None:
+            step.run_prefill()
+        if step.decode_cfg is not None:
+            step.run_decode()
+        for n, t in outs.items():
+            t.copy_(step.dev[n], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    secs = max_over_ranks(a.elapsed_time(b) / 1e3, world, device)
+    ideal = sum_over_ranks(step.ideal_seconds(peaks) * steps, world, device)
+    return {"value": ideal / secs, "unit": unit_string(), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps, "ms_per_step": 1e3 * secs / steps}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="default",
+                    choices=["default", "causal_mha", "causal_gqa", "long_causal", "tiny", "paged_decode"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line))
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, world, rank, local_rank)
+        if rank == 0:
+            print(json.dumps(line))
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,148 @@
+/*
+ * attn_b200.h -- C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * Two operations, both exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T + M) V,   LSE = log sum_j exp(scale * q . k_j)
+ * as defined in "Fast Attention Kernels and Operator Fusion" (wpnews.pro),
+ * section "FlashAttention-Style Kernels" (the attention equation with an
+ * additive mask M; is_causal=True makes M = -inf above the diagonal), fused so
+ * that the score matrix never reaches HBM; and its decode form over a paged KV
+ * cache read through a block table (same page, section "Paged Attention
+ * Kernels").
+ *
+ * Conventions for every entry point
+ *   - bf16 tensors are passed as pointers to raw bfloat16 bits (attn_bf16);
+ *     all tensor pointers are DEVICE pointers owned by the caller, 16-byte
+ *     aligned, contiguous, and must stay valid until the work queued on
+ *     `stream` has finished.  The library never frees or retains them.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream) of the current
+ *     device.  Calls only enqueue work: they never synchronise, never allocate
+ *     device memory, and return before the kernels run.
+ *   - The return value is an attn_status.  Argument errors are detected on the
+ *     host before anything is enqueued.  There is no fallback path: an
+ *     unsupported input is an error, never a slower kernel.  Errors raised
+ *     while the kernels run (a broken pipeline wait, a block-table entry
+ *     outside the pool) are recorded in a device error word that
+ *     attn_device_status() reads.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t attn_bf16; /* raw IEEE bfloat16 bits */
+
+typedef enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_NULL = 1,        /* a required pointer is NULL */
+  ATTN_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
+  ATTN_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  ATTN_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
+  ATTN_ERR_UNSUPPORTED = 5, /* valid input this build has no kernel for */
+  ATTN_ERR_LAUNCH = 6,      /* CUDA refused the launch (see attn_last_cuda_error) */
+  ATTN_ERR_DEVICE = 7       /* a kernel recorded a runtime error (attn_device_status) */
+} attn_status;
+
+/* Version of this ABI; bumped when a signature or a semantic changes. */
+int attn_abi_version(void);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char* attn_status_string(int status);
+
+/* The cudaError_t of the last failed CUDA call made by this library on the
+ * calling thread (0 if none). */
+int attn_last_cuda_error(void);
+
+/*
+ * attn_fwd -- fused attention forward (prefill).
+ *
+ *   q    [B, Hq,  N, d] bf16      queries
+ *   k    [B, Hkv, N, d] bf16      keys
+ *   v    [B, Hkv, N, d] bf16      values
+ *   o    [B, Hq,  N, d] bf16      output (written), rounded to nearest-even
+ *   lse  [B, Hq,  N]    float32   natural-log log-sum-exp of each row's scaled
+ *                                 scores over its visible keys (written)
+ *   d in {64, 128}; Hq % Hkv == 0, query head h reads KV head h / (Hq / Hkv)
+ *   causal: 0 = every key visible, 1 = query i sees keys j <= i
+ *   scale: multiplies Q K^T before the mask; must be finite and > 0
+ *
+ * Accumulation is fp32 (scores, softmax statistics, P V); P enters the second
+ * product as bf16.  o/lse may not alias q/k/v.
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE (sizes < 1, d not 64/128, Hq % Hkv,
+ * causal not 0/1, bad scale, a dimension too large for 32-bit indexing),
+ * ATTN_ERR_ALIGN, ATTN_ERR_LAUNCH.
+ */
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o,
+             float* lse, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+             void* stream);
+
+/*
+ * paged_attn_decode_split_tokens -- tokens per split of the split-KV decode
+ * pass for this problem shape (a multiple of 16).  The split plan depends only
+ * on these arguments, never on the sequence lengths, so the host never has to
+ * read device memory.
+ */
+int paged_attn_decode_split_tokens(int num_seqs, int Hkv, int max_pages, int page_size);
+
+/*
+ * paged_attn_decode_workspace_bytes -- bytes of device scratch that
+ * paged_attn_decode needs for these sizes: per (sequence, query head, split)
+ * a partial output row of d fp32 values and one fp32 partial LSE.  Returns 0
+ * for invalid sizes.
+ */
+size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_pages, int page_size);
+
+/*
+ * paged_attn_decode -- one-query-per-sequence attention over a paged KV cache.
+ *
+ *   q            [num_seqs, Hq, d] bf16       the newest token of each sequence
+ *   k_pool       [num_pages, page_size, Hkv, d] bf16
+ *   v_pool       [num_pages, page_size, Hkv, d] bf16
+ *   block_table  [num_seqs, max_pages] int32  logical page p of sequence s is
+ *                physical page block_table[s][p]; entries past a sequence's
+ *                ceil(seq_len / page_size) pages are never read (any value,
+ *                e.g. -1); entries may repeat across sequences (shared pages)
+ *   seq_lens     [num_seqs] int32, 1 <= seq_len <= max_pages * page_size; the
+ *                query attends to all seq_len cached tokens (no mask)
+ *   o            [num_seqs, Hq, d] bf16 (written)
+ *   lse          [num_seqs, Hq] float32, natural log (written)
+ *   page_size    a multiple of 16, at most 256
+ *   d in {64, 128}; Hq % Hkv == 0 and Hq / Hkv <= 16
+ *   workspace    device scratch of at least
+ *                paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_pages,
+ *                page_size) bytes, 16-byte aligned, owned by the caller; its
+ *                contents on entry do not matter; concurrent calls need
+ *                separate workspaces.
+ *
+ * Slots of a last page past seq_len may hold anything (NaN included) and do
+ * not affect the result.  A table entry outside [0, num_pages) or a length
+ * outside its range is reported through attn_device_status() (the affected
+ * outputs are then unspecified; invalid lengths give O = 0, LSE = -inf).
+ * Errors: ATTN_ERR_NULL, ATTN_ERR_SHAPE, ATTN_ERR_ALIGN, ATTN_ERR_WORKSPACE,
+ * ATTN_ERR_UNSUPPORTED (page_size, group size), ATTN_ERR_LAUNCH.
+ */
+int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                      const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                      attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
+                      int max_pages, int num_pages, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * attn_device_status -- synchronises `stream`, then reads and clears the
+ * device error word of the current device.  Returns ATTN_OK if no kernel
+ * recorded an error since the last call, ATTN_ERR_DEVICE otherwise (the raw
+ * bit mask is stored in *bits when bits != NULL), ATTN_ERR_LAUNCH if the
+ * synchronisation itself failed.
+ */
+int attn_device_status(void* stream, unsigned int* bits);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* ATTN_B200_H */

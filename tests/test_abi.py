@@ -1,0 +1,99 @@
+"""The C-ABI library: it loads, exports every declared symbol, and rejects bad
+arguments on the host before touching the GPU.  CPU only (no kernel runs:
+every call below fails validation before any CUDA call)."""
+
+import ctypes
+
+import pytest
+
+from attention_flashattention_fwd_04_b200 import api
+from attention_flashattention_fwd_04_b200.build import build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return api.lib()
+
+
+def test_every_declared_function_is_exported(lib):
+    names = api.header_functions()
+    assert set(names) == set(api.SIGNATURES), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.attn_abi_version() == 1
+    for code in range(8):
+        s = api.status_string(code)
+        assert s and s != "unknown status"
+    assert api.status_string(99) == "unknown status"
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null value; never dereferenced
+
+
+def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=16, d=64, causal=1,
+         scale=0.125):
+    return lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(o=None), 1), (dict(lse=None), 1),
+    (dict(B=0), 2), (dict(Hq=0), 2), (dict(Hkv=0), 2), (dict(N=0), 2), (dict(N=-5), 2),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(Hq=6, Hkv=4), 2), (dict(causal=2), 2),
+    (dict(scale=0.0), 2), (dict(scale=-1.0), 2), (dict(scale=float("inf")), 2), (dict(scale=float("nan")), 2),
+    (dict(B=1 << 16, Hq=1 << 16, Hkv=1 << 16), 2),
+    (dict(q=FAKE + 8), 3), (dict(o=FAKE + 2), 3), (dict(lse=FAKE + 2), 3),
+])
+def test_attn_fwd_rejects(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+def _dec(lib, q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, ps=16, o=FAKE, lse=FAKE, S=2, Hq=8, Hkv=2,
+         d=128, max_pages=4, num_pages=8, scale=0.1, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = lib.paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, ps) if ps > 0 else 0
+    return lib.paged_attn_decode(q, kp, vp, bt, sl, ps, o, lse, S, Hq, Hkv, d, max_pages, num_pages,
+                                 scale, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(kp=None), 1), (dict(vp=None), 1), (dict(bt=None), 1), (dict(sl=None), 1),
+    (dict(o=None), 1), (dict(lse=None), 1),
+    (dict(S=0), 2), (dict(Hq=0), 2), (dict(d=80), 2), (dict(Hq=6, Hkv=4), 2), (dict(max_pages=0), 2),
+    (dict(num_pages=0), 2), (dict(ps=0), 2), (dict(scale=0.0), 2), (dict(S=70000), 2),
+    (dict(ps=8), 5), (dict(ps=24), 5), (dict(ps=512), 5), (dict(Hq=34, Hkv=2), 5),
+    (dict(ws=None), 4), (dict(ws_bytes=16), 4),
+    (dict(q=FAKE + 4), 3), (dict(ws=FAKE + 8), 3), (dict(bt=FAKE + 2), 3),
+])
+def test_paged_decode_rejects(lib, kw, code):
+    assert _dec(lib, **kw) == code
+
+
+def test_workspace_formula(lib):
+    S, Hq, d, max_pages, ps = 64, 32, 128, 512, 16
+    split = lib.paged_attn_decode_split_tokens(S, 8, max_pages, ps)
+    assert split % 16 == 0 and split > 0
+    splits = -(-max_pages * ps // split)
+    rows = S * Hq * splits
+    o_bytes = rows * d * 4
+    lse_off = (o_bytes + 255) // 256 * 256
+    assert lib.paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, ps) == lse_off + rows * 4
+    assert lib.paged_attn_decode_workspace_bytes(0, Hq, d, max_pages, ps) == 0
+    assert lib.paged_attn_decode_workspace_bytes(S, Hq, 96, max_pages, ps) == 0
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        api.attn_fwd(q, q, q)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(api, "_lib", None)
+    monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        api.lib()
