@@ -43,8 +43,13 @@ SIGNATURES = {
     "paged_attn_decode_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
     "paged_attn_decode": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i,
                                  _c_i, _c_i, _c_f, _c_p, _c_sz, _c_p]),
+    "paged_attn_decode_noalloc": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_i, _c_i, _c_i,
+                                         _c_i, _c_i, _c_i, _c_f, _c_p]),
     "attn_device_status": (_c_i, [_c_p, ctypes.POINTER(ctypes.c_uint)]),
 }
+
+# Size of the scratch array built into the library for paged_attn_decode_noalloc.
+NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
 _lib = None
 
@@ -183,6 +188,40 @@ def paged_attn_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tenso
         page_size, out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages, float(scale),
         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _check(rc, "paged_attn_decode")
+    return out, lse
+
+
+def paged_attn_decode_noalloc(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                              block_table: torch.Tensor, seq_lens: torch.Tensor, scale: float | None = None,
+                              out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """paged_attn_decode without a workspace, for callers that may not
+    allocate device memory (the outputs still come from the caller; pass
+    ``out``/``lse`` to avoid any allocation here too).  The split partials go
+    to a 48 MiB array built into the library, shared by all calls on a
+    device: calls that can overlap on the GPU must not use it concurrently.
+    """
+    _require(q, "q", torch.bfloat16, 3)
+    _require(k_pool, "k_pool", torch.bfloat16, 4)
+    _require(v_pool, "v_pool", torch.bfloat16, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(seq_lens, "seq_lens", torch.int32, 1)
+    S, Hq, d = q.shape
+    num_pages, page_size, Hkv, _ = k_pool.shape
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    rc = lib().paged_attn_decode_noalloc(
+        q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+        page_size, out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, block_table.shape[1], num_pages,
+        float(scale), _stream_handle(stream))
+    if rc == 4:
+        need = paged_attn_decode_workspace_bytes(S, Hq, d, block_table.shape[1], page_size)
+        raise AttnError(rc, f"paged_attn_decode_noalloc: needs {need} bytes of scratch, "
+                            f"more than the built-in {NOALLOC_SCRATCH_BYTES}")
+    _check(rc, "paged_attn_decode_noalloc")
     return out, lse
 
 

@@ -133,6 +133,47 @@ int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf
                       size_t workspace_bytes, void* stream);
 
 /*
+ * ATTN_NOALLOC_SCRATCH_BYTES -- size of the device scratch array built into
+ * the library for paged_attn_decode_noalloc (48 MiB).
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+
+/*
+ * paged_attn_decode_noalloc -- paged_attn_decode for callers that cannot
+ * allocate device memory.  The pages have no counterpart to this call: it is
+ * a deployment convenience, not part of the method.
+ *
+ * Who needs it: a plug-in whose host program owns all device memory and does
+ * not let plug-ins allocate; a latency-critical serving loop, where a
+ * cudaMalloc may synchronise the device and stall other streams; a process
+ * whose memory pool has already reserved everything.  Such callers pass the
+ * same arguments as to paged_attn_decode minus the workspace, and the split
+ * partials go to a fixed array of ATTN_NOALLOC_SCRATCH_BYTES compiled into
+ * the library.  This call itself never allocates or frees device memory.
+ *
+ * - Every GPU on which the library's device code is loaded keeps that array
+ *   (48 MiB) until the process exits.
+ * - Limit: sizes whose paged_attn_decode_workspace_bytes() exceed
+ *   ATTN_NOALLOC_SCRATCH_BYTES are refused with ATTN_ERR_WORKSPACE before any
+ *   CUDA call.  (The 64-sequence, 32-head, 8192-token-table workload needs
+ *   33.8 MB.)
+ * - The first call with a given device current looks up the array's device
+ *   address (cudaGetSymbolAddress); make that first call before any stream
+ *   capture on that device.
+ * - All calls on a device share the one array and it keeps whatever the last
+ *   call left there (nothing in it needs to start at zero).  Calls whose
+ *   kernels can overlap on the GPU (different streams, or different host
+ *   threads without ordering) race on it and produce wrong results: order
+ *   them on one stream, or use paged_attn_decode with separate workspaces.
+ * Errors: those of paged_attn_decode, with ATTN_ERR_WORKSPACE meaning "larger
+ * than the built-in scratch".
+ */
+int paged_attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                              const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                              attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
+                              int max_pages, int num_pages, float scale, void* stream);
+
+/*
  * attn_device_status -- synchronises `stream`, then reads and clears the
  * device error word of the current device.  Returns ATTN_OK if no kernel
  * recorded an error since the last call, ATTN_ERR_DEVICE otherwise (the raw
