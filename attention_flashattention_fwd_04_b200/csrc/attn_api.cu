@@ -61,16 +61,31 @@ bool encode_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint
 bool misaligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kPrefillStages = 2;
+
+int sm_count() {
+  static int counts[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 0 || dev >= 64) return 0;
+  if (counts[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    counts[dev] = n;
+  }
+  return counts[dev];
+}
 
 template <int D, bool CAUSAL>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const attn::PrefillParams& p, cudaStream_t stream) {
-  using L = attn::PrefillLayout<D, kPrefillStages>;
-  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, kPrefillStages>;
+  using L = attn::PrefillLayout<D>;
+  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return fail_cuda(e);
-  const unsigned grid = static_cast<unsigned>(p.num_q_tiles) * static_cast<unsigned>(p.B * p.Hq);
+  const int sms = sm_count();
+  if (sms <= 0) return fail_cuda(cudaErrorInvalidDevice);
+  // Persistent: one CTA per SM (or per work item when there are fewer).
+  const unsigned grid = static_cast<unsigned>(p.num_items < sms ? p.num_items : sms);
   kernel<<<grid, attn::kPrefillThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail_cuda(e);
@@ -176,8 +191,8 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
   if (causal != 0 && causal != 1) return ATTN_ERR_SHAPE;
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_SHAPE;
   const long long bh = static_cast<long long>(B) * Hq;
-  const long long tiles = (static_cast<long long>(N) + 127) / 128;
-  if (bh > INT_MAX || tiles * bh > INT_MAX) return ATTN_ERR_SHAPE;
+  const long long blocks = (static_cast<long long>(N) + 255) / 256;
+  if (bh > INT_MAX || blocks * bh > INT_MAX) return ATTN_ERR_SHAPE;
   if (misaligned16(q) || misaligned16(k) || misaligned16(v) || misaligned16(o) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
     return ATTN_ERR_ALIGN;
@@ -198,7 +213,8 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
   p.Hkv = Hkv;
   p.N = N;
   p.group = Hq / Hkv;
-  p.num_q_tiles = static_cast<int>(tiles);
+  p.num_m = static_cast<int>(blocks);
+  p.num_items = static_cast<int>(blocks * bh);
   p.scale_log2 = scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 128)

@@ -323,6 +323,8 @@ __global__ void __launch_bounds__(32 * (HB + 1), 1)
 }
 
 // One warp per (sequence, query head): combine the splits that hold tokens.
+// Lane i computes the weight of split i of each group of 32; the partial rows
+// are then read eight splits at a time so that eight loads are in flight.
 template <int D>
 __global__ void __launch_bounds__(256)
     decode_merge_kernel(const DecodeParams p, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
@@ -341,29 +343,53 @@ __global__ void __launch_bounds__(256)
   }
   const int n_splits = (seq_len + p.split_tokens - 1) / p.split_tokens;
   const float* plse = p.part_lse + static_cast<size_t>(wid) * p.max_splits;
-  const float* po = p.part_o + static_cast<size_t>(wid) * p.max_splits * D;
+  const float* po = p.part_o + static_cast<size_t>(wid) * p.max_splits * D + lane * kPer;
   constexpr float kLog2e = 1.4426950408889634f;
   float mx = -INFINITY;
   for (int t = lane; t < n_splits; t += 32) mx = fmaxf(mx, plse[t]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   float wsum = 0.f;
-  for (int t = lane; t < n_splits; t += 32) wsum += ex2_approx((plse[t] - mx) * kLog2e);
+  float out[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) out[e] = 0.f;
+  for (int t0 = 0; t0 < n_splits; t0 += 32) {
+    const int cnt = min(32, n_splits - t0);
+    const float my_w = lane < cnt ? ex2_approx((plse[t0 + lane] - mx) * kLog2e) : 0.f;
+    wsum += my_w;
+    for (int i = 0; i < cnt; i += 8) {
+      float v[8][kPer];
+      float w[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        w[u] = __shfl_sync(0xffffffffu, my_w, (i + u) & 31);
+        if (i + u < cnt) {
+          const float* src = po + static_cast<size_t>(t0 + i + u) * D;
+          if constexpr (kPer == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(src);
+            v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+          } else {
+            const float2 x = *reinterpret_cast<const float2*>(src);
+            v[u][0] = x.x; v[u][1] = x.y;
+          }
+        } else {
+          w[u] = 0.f;
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) v[u][e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) out[e] = fmaf(w[u], v[u][e], out[e]);
+    }
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
   const float inv = 1.f / wsum;
-  float out[kPer];
 #pragma unroll
-  for (int i = 0; i < kPer; ++i) out[i] = 0.f;
-  for (int t = 0; t < n_splits; ++t) {
-    const float w = ex2_approx((plse[t] - mx) * kLog2e) * inv;
-    const float* src = po + static_cast<size_t>(t) * D + lane * kPer;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) out[i] = fmaf(w, src[i], out[i]);
-  }
-#pragma unroll
-  for (int i = 0; i < kPer; i += 2)
-    *reinterpret_cast<uint32_t*>(orow + lane * kPer + i) = pack_bf16x2(out[i], out[i + 1]);
+  for (int e = 0; e < kPer; e += 2)
+    *reinterpret_cast<uint32_t*>(orow + lane * kPer + e) = pack_bf16x2(out[e] * inv, out[e + 1] * inv);
   if (lane == 0) lse[wid] = mx + logf(wsum);
 }
 
