@@ -28,10 +28,36 @@
 // place without a further wait.
 #pragma once
 
+#include "exp2_poly.cuh"
 #include "ptx.cuh"
 #include "tmem_ldst.cuh"
 
 namespace attn {
+
+// One column pair in every kExp2EmuPeriod takes its exp2 from a polynomial on
+// the FMA pipes instead of the MUFU unit, which is otherwise as busy as the
+// tensor core (0 disables it).
+#ifndef ATTN_EXP2_EMU_PERIOD
+#define ATTN_EXP2_EMU_PERIOD 0
+#endif
+constexpr int kExp2EmuPeriod = ATTN_EXP2_EMU_PERIOD;
+
+
+
+// 2^x by range reduction x = n + f, n = round(x), |f| <= 1/2: adding
+// 1.5*2^23 rounds x to an integer held in the low mantissa bits, 2^f comes
+// from the fitted cubic (exp2_poly.cuh) and n is added to the exponent field.
+// x is clamped at -126 so the exponent never underflows past zero.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float q = fmaf(kExp2C3, f, kExp2C2);
+  q = fmaf(q, f, kExp2C1);
+  q = fmaf(q, f, kExp2C0);
+  // (bits(t) - bits(1.5*2^23)) << 23 == bits(t) << 23: the constant's low 9 bits are 0.
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
 
 struct PrefillParams {
   __nv_bfloat16* o;  // [B, Hq, N, D]
@@ -113,15 +139,15 @@ __device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, 
 }
 
 // Register split per warpgroup (launch: 512 threads x 128 registers):
-// softmax 2 x 176, epilogue 72, producer/MMA 88 -> 4 x 128 per lane slot.
+// softmax 2 x 184, epilogue 64, producer/MMA 80 -> 4 x 128 per lane slot.
 __device__ __forceinline__ void reg_alloc_softmax() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 176;\n" ::: "memory");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 184;\n" ::: "memory");
 }
 __device__ __forceinline__ void reg_alloc_epilogue() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
 }
 __device__ __forceinline__ void reg_alloc_control() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 88;\n" ::: "memory");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
 }
 
 template <int D, bool CAUSAL>
@@ -282,7 +308,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const uint32_t ph = static_cast<uint32_t>(g / NS) & 1u, ph1 = static_cast<uint32_t>((g + 1) / NS) & 1u;
           bool v_ready = false, k_ready = false;
           if (j < it.n0) {
-            if (!(ok = mbar_wait(bar(L::kBarPFull + 0), p_cnt[0]++ & 1u, kErrWaitPFull))) break;
+            const uint32_t pph = p_cnt[0]++ & 1u;
+            if (!(ok = mbar_wait(bar(L::kBarPFull + 0), pph, kErrWaitPFull))) break;
             if (j == 0 && r > 0 &&
                 !(ok = mbar_wait(bar(L::kBarOFree), static_cast<uint32_t>(r - 1) & 1u, kErrWaitODone)))
               break;
@@ -298,7 +325,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
           }
           if (j < it.n1) {
-            if (!(ok = mbar_wait(bar(L::kBarPFull + 1), p_cnt[1]++ & 1u, kErrWaitPFull))) break;
+            const uint32_t pph = p_cnt[1]++ & 1u;
+            if (!(ok = mbar_wait(bar(L::kBarPFull + 1), pph, kErrWaitPFull))) break;
             if (!v_ready && !(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
             tc_fence_after();
             issue_pv(1, st, j > 0);
@@ -350,19 +378,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const size_t row_index = static_cast<size_t>(it.b * p.Hq + it.h) * p.N + grow;
         __nv_bfloat16* orow = p.o + row_index * D;
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          tmem_ld_x32_wait(lane_addr + L::kColO + static_cast<uint32_t>(t * D + c), o);
-          uint32_t w[16];
+        for (int c = 0; c < D; c += 16) {
+          uint32_t o[16];
+          tmem_ld_x16_wait(lane_addr + L::kColO + static_cast<uint32_t>(t * D + c), o);
+          uint32_t w[8];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < 8; ++i)
             w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
           if (grow < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
-            dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
           }
         }
         if (grow < p.N) p.lse[row_index] = (m_used + log2f(l_sum)) * kLn2;
@@ -406,59 +432,70 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           for (int c = 0; c < 128; ++c)
             if (kv0 + c > last) s[c] = -INFINITY;
         }
+        // Row max: four chains of three-input maxima.
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 4; c < 128; c += 8) {
+          mx0 = max3(mx0, s[c], s[c + 1]);
+          mx1 = max3(mx1, s[c + 2], s[c + 3]);
+          mx2 = max3(mx2, s[c + 4], s[c + 5]);
+          mx3 = max3(mx3, s[c + 6], s[c + 7]);
         }
-        const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        m_tile *= sl2;
         const float m_new = fmaxf(m_used, m_tile);
         const bool upd = m_new > m_used + kRescaleThreshold;
         const float alpha = upd ? ex2_approx(m_used - m_new) : 1.f;  // 0 on the first tile
         if (upd) m_used = m_new;
         l_sum *= alpha;
         const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
-        uint32_t pk_lo[32], pk_hi[32];
-        float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        const uint64_t negm2 = f2_pack(neg_m, neg_m);
+        // P in two halves, columns [0, 64) then [64, 128); each half goes to
+        // tensor memory as soon as it is packed (fewer live registers).
+        uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) {
-          const float p0 = ex2_approx(fmaf(s[c], sl2, neg_m));
-          const float p1 = ex2_approx(fmaf(s[c + 1], sl2, neg_m));
-          const float p2 = ex2_approx(fmaf(s[c + 2], sl2, neg_m));
-          const float p3 = ex2_approx(fmaf(s[c + 3], sl2, neg_m));
-          ls0 += p0;
-          ls1 += p1;
-          ls2 += p2;
-          ls3 += p3;
-          if (c < 64) {
-            pk_lo[c / 2] = pack_bf16x2(p0, p1);
-            pk_lo[c / 2 + 1] = pack_bf16x2(p2, p3);
-          } else {
-            pk_hi[(c - 64) / 2] = pack_bf16x2(p0, p1);
-            pk_hi[(c - 64) / 2 + 1] = pack_bf16x2(p2, p3);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int c = half * 64 + 2 * i;
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2), x0, x1);
+            float p0, p1;
+            if (kExp2EmuPeriod > 0 && i % (kExp2EmuPeriod > 0 ? kExp2EmuPeriod : 1) == kExp2EmuPeriod - 1) {
+              p0 = exp2_poly(x0);
+              p1 = exp2_poly(x1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            acc[i & 1] = f2_add(acc[i & 1], f2_pack(p0, p1));
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_x32(s_addr + static_cast<uint32_t>(half * 32), pk);
+          if (half == 0 && j > 0 && __any_sync(0xffffffffu, upd)) {
+            // O_t is idle here (its last update was issued before S_t of this
+            // tile, and this tile's update waits for the barrier below).
+#pragma unroll
+            for (int c = 0; c < D; c += 32) {
+              uint32_t o[32];
+              tmem_ld_x32_wait(o_addr + c, o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st_x32(o_addr + c, o);
+            }
+          }
+          if (half == 1) {
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(L::kBarPFull + t));
           }
         }
+        float ls0, ls1, ls2, ls3;
+        f2_unpack(acc[0], ls0, ls1);
+        f2_unpack(acc[1], ls2, ls3);
         l_sum += (ls0 + ls1) + (ls2 + ls3);
-        tmem_st_x32(s_addr, pk_lo);
-        tmem_st_x32(s_addr + 32u, pk_hi);
-        // Rescale after P is out (the scores are dead by now); O_t is idle
-        // here: its last update was issued before S_t of this tile.
-        if (j > 0 && __any_sync(0xffffffffu, upd)) {
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            tmem_ld_x32_wait(o_addr + c, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_x32(o_addr + c, o);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(L::kBarPFull + t));
       }
       if (!ok) break;
       // Hand m and l of this row to the epilogue (2-slot ring per tile).
