@@ -93,9 +93,9 @@ struct PrefillLayout {
   static constexpr int kBarVEmpty = kBarVFull + NS;
   static constexpr int kBarSFull = kBarVEmpty + NS;     // [tile]
   static constexpr int kBarPFull = kBarSFull + 2;       // [tile]
-  static constexpr int kBarOFull = kBarPFull + 2;
-  static constexpr int kBarOFree = kBarOFull + 1;
-  static constexpr int kBarStatsFull = kBarOFree + 1;   // [tile][slot]
+  static constexpr int kBarOFull = kBarPFull + 2;       // [tile]: O_t of the item is final
+  static constexpr int kBarOFree = kBarOFull + 2;       // [tile]: the epilogue has read O_t
+  static constexpr int kBarStatsFull = kBarOFree + 2;   // [tile][slot]
   static constexpr int kBarStatsEmpty = kBarStatsFull + 4;
   static constexpr int kBarMmaDone = kBarStatsEmpty + 4;
   static constexpr int kNumBars = kBarMmaDone + 1;
@@ -182,8 +182,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar(L::kBarSFull + t), 1);
       mbar_init(bar(L::kBarPFull + t), 128);
     }
-    mbar_init(bar(L::kBarOFull), 1);
-    mbar_init(bar(L::kBarOFree), 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::kBarOFull + t), 1);
+      mbar_init(bar(L::kBarOFree + t), 128);
+    }
     for (int i = 0; i < 4; ++i) {
       mbar_init(bar(L::kBarStatsFull + i), 128);
       mbar_init(bar(L::kBarStatsEmpty + i), 128);
@@ -267,6 +269,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, false, true);
       int kv_it = 0;
       uint32_t p_cnt[2] = {0u, 0u};
+      uint32_t o_cnt[2] = {0u, 0u};  // items whose O_t has been completed
       bool ok = true;
       auto issue_s = [&](int t, int st) {
         const uint32_t q_addr = base + (t ? L::kQ1 : L::kQ0);
@@ -310,13 +313,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (j < it.n0) {
             const uint32_t pph = p_cnt[0]++ & 1u;
             if (!(ok = mbar_wait(bar(L::kBarPFull + 0), pph, kErrWaitPFull))) break;
-            if (j == 0 && r > 0 &&
-                !(ok = mbar_wait(bar(L::kBarOFree), static_cast<uint32_t>(r - 1) & 1u, kErrWaitODone)))
+            if (j == 0 && o_cnt[0] > 0 &&
+                !(ok = mbar_wait(bar(L::kBarOFree + 0), (o_cnt[0] - 1u) & 1u, kErrWaitODone)))
               break;
             if (!(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
             v_ready = true;
             tc_fence_after();
             issue_pv(0, st, j > 0);
+            if (j + 1 == it.n0) {
+              mma_commit(bar(L::kBarOFull + 0));  // O0 of this item is final once this lands
+              ++o_cnt[0];
+            }
             if (j + 1 < it.n0) {
               if (!(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
               k_ready = true;
@@ -327,9 +334,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (j < it.n1) {
             const uint32_t pph = p_cnt[1]++ & 1u;
             if (!(ok = mbar_wait(bar(L::kBarPFull + 1), pph, kErrWaitPFull))) break;
+            if (j == 0 && o_cnt[1] > 0 &&
+                !(ok = mbar_wait(bar(L::kBarOFree + 1), (o_cnt[1] - 1u) & 1u, kErrWaitODone)))
+              break;
             if (!v_ready && !(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
             tc_fence_after();
             issue_pv(1, st, j > 0);
+            if (j + 1 == it.n1) {
+              mma_commit(bar(L::kBarOFull + 1));
+              ++o_cnt[1];
+            }
             if (j + 1 < it.n1) {
               if (!k_ready && !(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
               tc_fence_after();
@@ -341,7 +355,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (j + 2 == it.n_kv) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
         }
         if (!ok) break;
-        mma_commit(bar(L::kBarOFull));
         kv_it += it.n_kv;
       }
       // All issued MMAs must finish before tensor memory is released.
@@ -354,20 +367,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     reg_alloc_epilogue();
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    uint32_t st_cnt[2] = {0u, 0u};
+    uint32_t st_cnt[2] = {0u, 0u};  // items whose tile t this warpgroup has written out
     bool ok = true;
     PrefillItem it;
     for (int r = 0; ok && prefill_item<CAUSAL>(r, p, it); ++r) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarOFull), static_cast<uint32_t>(r) & 1u, kErrWaitODone));
-      if (!ok) break;
-      tc_fence_after();
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if ((t == 0 ? it.n0 : it.n1) == 0) continue;
-        const uint32_t slot = st_cnt[t] & 1u;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStatsFull + 2 * t + slot), (st_cnt[t] >> 1) & 1u,
+        const uint32_t n = st_cnt[t];
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarOFull + t), n & 1u, kErrWaitODone));
+        if (!ok) break;
+        const uint32_t slot = n & 1u;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarStatsFull + 2 * t + slot), (n >> 1) & 1u,
                                                kErrWaitSFull));
         if (!ok) break;
+        tc_fence_after();
         const float* sp = stats + ((t * 2 + slot) * 2) * 128;
         const float m_used = sp[row];
         const float l_sum = sp[128 + row];
@@ -378,24 +392,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const size_t row_index = static_cast<size_t>(it.b * p.Hq + it.h) * p.N + grow;
         __nv_bfloat16* orow = p.o + row_index * D;
 #pragma unroll
-        for (int c = 0; c < D; c += 16) {
-          uint32_t o[16];
-          tmem_ld_x16_wait(lane_addr + L::kColO + static_cast<uint32_t>(t * D + c), o);
-          uint32_t w[8];
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld_x32_wait(lane_addr + L::kColO + static_cast<uint32_t>(t * D + c), o);
+          uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+          for (int i = 0; i < 16; ++i)
             w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
           if (grow < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            dst[2] = make_uint4(w[8], w[9], w[10], w[11]);
+            dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
           }
         }
         if (grow < p.N) p.lse[row_index] = (m_used + log2f(l_sum)) * kLn2;
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarOFree + t));
       }
-      if (!ok) break;
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarOFree));
     }
   } else {
     // ------------------------------------------------------------ softmax (tile t = wg)
