@@ -484,9 +484,13 @@ def run_ours(args, world, rank, local_rank):
     dominant = max(kernels, key=lambda k: kernels[k]["us_per_launch"])
     traffic = load_traffic()
     dk = kernels[dominant]
-    tkey = "prefill_fwd_kernel" if dominant.startswith("prefill") else "decode_split_kernel"
+    if dominant.startswith("prefill"):
+        tr = traffic.get("prefill_fwd_kernel")
+    else:
+        parts = [traffic.get("decode_split_kernel"), traffic.get("decode_merge_kernel")]
+        tr = None if any(x is None for x in parts) else sum(parts)
     line["roofline"] = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
-                        "unit": dk["unit"], "frac": dk["frac"], "traffic": traffic.get(tkey),
+                        "unit": dk["unit"], "frac": dk["frac"], "traffic": tr,
                         "peak_source": f"{peaks['source']} (burst)"}
     line["kernels"] = kernels
     line["e2e"] = e2e
