@@ -45,6 +45,11 @@ SIGNATURES = {
                                  _c_i, _c_i, _c_f, _c_p, _c_sz, _c_p]),
     "paged_attn_decode_noalloc": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_i, _c_i, _c_i,
                                          _c_i, _c_i, _c_i, _c_f, _c_p]),
+    "paged_attn_decode_graph_create": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_i, _c_i, _c_i,
+                                              _c_i, _c_i, _c_i, _c_f, _c_p, _c_sz,
+                                              ctypes.POINTER(ctypes.c_void_p)]),
+    "paged_attn_decode_graph_launch": (_c_i, [_c_p, _c_p]),
+    "paged_attn_decode_graph_destroy": (_c_i, [_c_p]),
     "attn_device_status": (_c_i, [_c_p, ctypes.POINTER(ctypes.c_uint)]),
 }
 
@@ -223,6 +228,59 @@ def paged_attn_decode_noalloc(q: torch.Tensor, k_pool: torch.Tensor, v_pool: tor
                             f"more than the built-in {NOALLOC_SCRATCH_BYTES}")
     _check(rc, "paged_attn_decode_noalloc")
     return out, lse
+
+
+class DecodeGraph:
+    """One paged-decode step (split pass + merge) captured as a CUDA graph.
+
+    Construct it with the same tensors as :func:`paged_attn_decode`; then
+    change their contents in place (same shapes) and call :meth:`launch` for
+    each step.  The tensors, the workspace and the outputs are kept alive by
+    this object; ``out`` and ``lse`` hold the results after each launch.
+    """
+
+    def __init__(self, q, k_pool, v_pool, block_table, seq_lens, scale=None, workspace=None, out=None, lse=None):
+        for t, name, dt, nd in ((q, "q", torch.bfloat16, 3), (k_pool, "k_pool", torch.bfloat16, 4),
+                                (v_pool, "v_pool", torch.bfloat16, 4), (block_table, "block_table", torch.int32, 2),
+                                (seq_lens, "seq_lens", torch.int32, 1)):
+            _require(t, name, dt, nd)
+        S, Hq, d = q.shape
+        num_pages, page_size, Hkv, _ = k_pool.shape
+        max_pages = block_table.shape[1]
+        if scale is None:
+            scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+        need = paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, page_size)
+        self.workspace = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8,
+                                                                             device=q.device)
+        self.out = out if out is not None else torch.empty_like(q)
+        self.lse = lse if lse is not None else torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+        self._keep = (q, k_pool, v_pool, block_table, seq_lens)
+        handle = ctypes.c_void_p()
+        rc = lib().paged_attn_decode_graph_create(
+            q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+            page_size, self.out.data_ptr(), self.lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages,
+            float(scale), self.workspace.data_ptr(), self.workspace.numel() * self.workspace.element_size(),
+            ctypes.byref(handle))
+        _check(rc, "paged_attn_decode_graph_create")
+        self._handle = handle
+
+    def launch(self, stream=None):
+        if self._handle is None:
+            raise RuntimeError("DecodeGraph is closed")
+        _check(lib().paged_attn_decode_graph_launch(self._handle, _stream_handle(stream)),
+               "paged_attn_decode_graph_launch")
+        return self.out, self.lse
+
+    def close(self):
+        h, self._handle = getattr(self, "_handle", None), None
+        if h is not None:
+            _check(lib().paged_attn_decode_graph_destroy(h), "paged_attn_decode_graph_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def device_status(stream=None) -> int:

@@ -5,10 +5,12 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <new>
 
 #include "attn_b200.h"
 #include "decode_sm100.cuh"
@@ -60,6 +62,21 @@ bool encode_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint
 
 bool misaligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
+// Raises a kernel's dynamic shared-memory limit once per device (the
+// attribute is per device), so launches do not repeat the driver call.
+template <auto Kernel>
+cudaError_t ensure_smem_limit(int bytes) {
+  static std::atomic<uint64_t> done{0};  // one bit per device ordinal < 64
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit != 0) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 
 int sm_count() {
@@ -80,7 +97,7 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
                    const attn::PrefillParams& p, cudaStream_t stream) {
   using L = attn::PrefillLayout<D>;
   auto kernel = attn::prefill_fwd_kernel<D, CAUSAL>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL>>(L::kAlloc);
   if (e != cudaSuccess) return fail_cuda(e);
   const int sms = sm_count();
   if (sms <= 0) return fail_cuda(cudaErrorInvalidDevice);
@@ -98,12 +115,25 @@ int decode_heads_per_cta(int Hkv) {
   return hb;
 }
 
+// The split plan depends only on sizes (the lengths live on the device): 256
+// tokens per split, halved (down to 64) while a full-length batch would give
+// fewer than kDecodeTargetCtas CTAs, so small batches still fill the GPU.
+constexpr long long kDecodeTargetCtas = 2 * 148;
+
 int split_tokens_for(int num_seqs, int Hkv, int max_pages, int page_size) {
-  (void)num_seqs;
   (void)Hkv;
-  (void)max_pages;
-  (void)page_size;
-  return 256;
+  const long long max_tokens = static_cast<long long>(max_pages) * page_size;
+  long long split = 256;
+  while (split > 64 && num_seqs * ((max_tokens + split - 1) / split) < kDecodeTargetCtas) split /= 2;
+  return static_cast<int>(split);
+}
+
+// KV heads per CTA: up to 8 (one page chunk of all heads per TMA box pair),
+// fewer when that leaves too few CTAs.
+int decode_heads_for(int num_seqs, int Hkv, int max_splits) {
+  int hb = decode_heads_per_cta(Hkv);
+  while (hb > 1 && static_cast<long long>(num_seqs) * max_splits * (Hkv / hb) < kDecodeTargetCtas) hb /= 2;
+  return hb;
 }
 
 struct DecodePlan {
@@ -134,7 +164,7 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const attn::Deco
                   attn_bf16* o, float* lse, cudaStream_t stream) {
   using L = attn::DecodeLayout<D, HB>;
   auto split_kernel = attn::decode_split_kernel<D, HB>;
-  cudaError_t e = cudaFuncSetAttribute(split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  cudaError_t e = ensure_smem_limit<attn::decode_split_kernel<D, HB>>(L::kAlloc);
   if (e != cudaSuccess) return fail_cuda(e);
   const dim3 grid(static_cast<unsigned>(p.max_splits), static_cast<unsigned>(p.S),
                   static_cast<unsigned>(p.Hkv / HB));
@@ -232,11 +262,15 @@ size_t paged_attn_decode_workspace_bytes(int num_seqs, int Hq, int d, int max_pa
   return pl.total;
 }
 
-int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
-                      const int32_t* block_table, const int32_t* seq_lens, int page_size,
-                      attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
-                      int max_pages, int num_pages, float scale, void* workspace,
-                      size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Host-side argument checks of paged_attn_decode (no CUDA call).
+int validate_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                    const int32_t* block_table, const int32_t* seq_lens, int page_size, attn_bf16* o,
+                    float* lse, int num_seqs, int Hq, int Hkv, int d, int max_pages, int num_pages,
+                    float scale, void* workspace, size_t workspace_bytes, DecodePlan* plan) {
   if (!q || !k_pool || !v_pool || !block_table || !seq_lens || !o || !lse) return ATTN_ERR_NULL;
   if (num_seqs < 1 || Hq < 1 || Hkv < 1 || max_pages < 1 || num_pages < 1 || page_size < 1)
     return ATTN_ERR_SHAPE;
@@ -256,8 +290,26 @@ int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf
       (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(seq_lens) & 3u) != 0)
     return ATTN_ERR_ALIGN;
+  *plan = pl;
+  return ATTN_OK;
+}
 
-  const int hb = decode_heads_per_cta(Hkv);
+}  // namespace
+
+extern "C" {
+
+
+int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                      const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                      attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
+                      int max_pages, int num_pages, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  DecodePlan pl;
+  const int vs = validate_decode(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv,
+                                 d, max_pages, num_pages, scale, workspace, workspace_bytes, &pl);
+  if (vs != ATTN_OK) return vs;
+
+  const int hb = decode_heads_for(num_seqs, Hkv, pl.max_splits);
   CUtensorMap tk, tv;
   const uint64_t token_bytes = static_cast<uint64_t>(Hkv) * d * 2;
   const uint64_t head_bytes = static_cast<uint64_t>(d) * 2;
@@ -285,6 +337,102 @@ int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 128) return dispatch_decode_hb<128>(hb, tk, tv, p, o, lse, s);
   return dispatch_decode_hb<64>(hb, tk, tv, p, o, lse, s);
+}
+
+}  // extern "C"
+
+// A captured decode step: the split pass and the merge as one CUDA graph.
+struct attn_decode_graph {
+  cudaGraphExec_t exec = nullptr;
+  int device = -1;
+};
+
+namespace {
+
+// Everything a decode launch needs that is not a stream operation, done
+// before capture so that capture only records the two kernel launches.
+cudaError_t prepare_decode(int d, int Hkv, int num_seqs, int max_splits) {
+  if (!encode_fn()) return cudaErrorInvalidValue;
+  const int hb = decode_heads_for(num_seqs, Hkv, max_splits);
+  auto one = [&](auto tag) -> cudaError_t {
+    constexpr int D = decltype(tag)::value;
+    switch (hb) {
+      case 8: return ensure_smem_limit<attn::decode_split_kernel<D, 8>>(attn::DecodeLayout<D, 8>::kAlloc);
+      case 4: return ensure_smem_limit<attn::decode_split_kernel<D, 4>>(attn::DecodeLayout<D, 4>::kAlloc);
+      case 2: return ensure_smem_limit<attn::decode_split_kernel<D, 2>>(attn::DecodeLayout<D, 2>::kAlloc);
+      default: return ensure_smem_limit<attn::decode_split_kernel<D, 1>>(attn::DecodeLayout<D, 1>::kAlloc);
+    }
+  };
+  return d == 128 ? one(std::integral_constant<int, 128>{}) : one(std::integral_constant<int, 64>{});
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attn_decode_graph_create(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                                   const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                                   attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
+                                   int max_pages, int num_pages, float scale, void* workspace,
+                                   size_t workspace_bytes, attn_decode_graph** graph) {
+  if (!graph) return ATTN_ERR_NULL;
+  *graph = nullptr;
+  DecodePlan pl;
+  const int vs = validate_decode(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv,
+                                 d, max_pages, num_pages, scale, workspace, workspace_bytes, &pl);
+  if (vs != ATTN_OK) return vs;
+  {
+    const cudaError_t e = prepare_decode(d, Hkv, num_seqs, pl.max_splits);
+    if (e != cudaSuccess) return fail_cuda(e);
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail_cuda(e);
+  cudaStream_t s = nullptr;
+  e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return fail_cuda(e);
+  e = cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) {
+    cudaStreamDestroy(s);
+    return fail_cuda(e);
+  }
+  const int rc = paged_attn_decode(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq,
+                                   Hkv, d, max_pages, num_pages, scale, workspace, workspace_bytes, s);
+  cudaGraph_t g = nullptr;
+  const cudaError_t end = cudaStreamEndCapture(s, &g);
+  cudaStreamDestroy(s);
+  if (rc != ATTN_OK || end != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    return rc != ATTN_OK ? rc : fail_cuda(end);
+  }
+  cudaGraphExec_t exec = nullptr;
+  e = cudaGraphInstantiate(&exec, g, 0);
+  cudaGraphDestroy(g);
+  if (e != cudaSuccess) return fail_cuda(e);
+  attn_decode_graph* h = new (std::nothrow) attn_decode_graph;
+  if (!h) {
+    cudaGraphExecDestroy(exec);
+    return fail_cuda(cudaErrorMemoryAllocation);
+  }
+  h->exec = exec;
+  h->device = dev;
+  *graph = h;
+  return ATTN_OK;
+}
+
+int paged_attn_decode_graph_launch(attn_decode_graph* graph, void* stream) {
+  if (!graph || !graph->exec) return ATTN_ERR_NULL;
+  const cudaError_t e = cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail_cuda(e);
+  return ATTN_OK;
+}
+
+int paged_attn_decode_graph_destroy(attn_decode_graph* graph) {
+  if (!graph) return ATTN_OK;
+  cudaError_t e = cudaSuccess;
+  if (graph->exec) e = cudaGraphExecDestroy(graph->exec);
+  delete graph;
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(e);
 }
 
 int attn_device_status(void* stream, unsigned int* bits) {

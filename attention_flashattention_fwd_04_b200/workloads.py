@@ -93,6 +93,8 @@ PREFILL_CONFIGS = {
 
 DECODE_CONFIGS = {
     "paged_decode": DecodeConfig("paged_decode", 64, 32, 8, 128, 16, 512, 8192, 4),
+    # a small decode batch, where per-call host work and launch gaps dominate
+    "small_decode": DecodeConfig("small_decode", 4, 32, 8, 128, 16, 256, 1024, 6),
 }
 
 

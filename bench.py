@@ -13,7 +13,8 @@ i.e. the time-weighted fraction of the measured B200 peaks the step reaches
 separate prefill TFLOP/s and decode GB/s are in the line too.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--workload default|causal_mha|causal_gqa|long_causal|paged_decode]
+       [--workload default|causal_mha|causal_gqa|long_causal|paged_decode|small_decode]
+       [--decode-graph]
 Under torchrun each rank runs its own batch (seed offset by rank), no
 collective on the data path; rank 0 prints one JSON line.
 """
@@ -169,7 +170,7 @@ class ClockSampler:
 class Step:
     """Device-resident inputs/outputs for one rank and the calls of one step."""
 
-    def __init__(self, workload: str, rank: int, device):
+    def __init__(self, workload: str, rank: int, device, decode_graph: bool = False):
         from attention_flashattention_fwd_04_b200 import api
         self.api = api
         self.device = device
@@ -180,8 +181,8 @@ class Step:
             base = W.PREFILL_CONFIGS[name]
             self.prefill_cfg = W.PrefillConfig(base.name, base.B, base.Hq, base.Hkv, base.N, base.d, base.causal,
                                                shard_seed(base.seed, rank), base.value_scale, base.k_offset_sigma)
-        if workload in ("default", "paged_decode"):
-            base = W.DECODE_CONFIGS["paged_decode"]
+        if workload in ("default", "paged_decode", "small_decode"):
+            base = W.DECODE_CONFIGS["small_decode" if workload == "small_decode" else "paged_decode"]
             self.decode_cfg = W.DecodeConfig(base.name, base.num_seqs, base.Hq, base.Hkv, base.d, base.page_size,
                                              base.min_len, base.max_len, shard_seed(base.seed, rank))
         self.host = {}
@@ -203,6 +204,11 @@ class Step:
         for name, t in self.host.items():
             self.dev[name] = t.to(device)
         self._alloc_outputs()
+        self.graph = None
+        if decode_graph and self.decode_cfg is not None:
+            d = self.dev
+            self.graph = api.DecodeGraph(d["dq"], d["k_pool"], d["v_pool"], d["block_table"], d["seq_lens"],
+                                         self.decode_cfg.scale, workspace=d["ws"], out=d["do"], lse=d["dlse"])
 
     def _alloc_outputs(self):
         api, dev = self.api, self.device
@@ -227,6 +233,9 @@ class Step:
 
     def run_decode(self, d=None):
         d = d or self.dev
+        if self.graph is not None:
+            self.graph.launch()
+            return
         c = self.decode_cfg
         self.api.paged_attn_decode(d["dq"], d["k_pool"], d["v_pool"], d["block_table"], d["seq_lens"], c.scale,
                                    workspace=self.dev["ws"], out=d["do"], lse=d["dlse"])
@@ -252,6 +261,8 @@ def config_dict(step: Step, n_gpus: int):
                          "len_range": [c.min_len, c.max_len], "total_tokens": int(L.sum()),
                          "num_pages": step.decode_inp["num_pages"], "seed": c.seed, "bytes": step.bytes}
     cfg["workload"] = " + ".join(parts)
+    if step.graph is not None:
+        cfg["decode_graph"] = True
     if step.decode_cfg is not None:
         cfg["l2"] = "inputs larger than L2: the decode pass streams >1 GB of KV through the 126 MB L2 every step"
     else:
@@ -377,8 +388,8 @@ class StepHost:
             self.host.update(q=q, k=k, v=v)
             c = self.prefill_cfg
             parts.append(f"causal prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}")
-        if workload in ("default", "paged_decode"):
-            self.decode_cfg = W.DECODE_CONFIGS["paged_decode"]
+        if workload in ("default", "paged_decode", "small_decode"):
+            self.decode_cfg = W.DECODE_CONFIGS["small_decode" if workload == "small_decode" else "paged_decode"]
             inp = W.make_decode_inputs(self.decode_cfg)
             self.decode_inp = inp
             self.host.update(dq=inp["q"], k_pool=inp["k_pool"], v_pool=inp["v_pool"],
@@ -400,7 +411,7 @@ def run_ours(args, world, rank, local_rank):
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     peaks = load_peaks()
-    step = Step(args.workload, rank, device)
+    step = Step(args.workload, rank, device, decode_graph=args.decode_graph)
     stream = torch.cuda.current_stream()
     flush = None
     if step.decode_cfg is None:
@@ -556,7 +567,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="default",
-                    choices=["default", "causal_mha", "causal_gqa", "long_causal", "tiny", "paged_decode"])
+                    choices=["default", "causal_mha", "causal_gqa", "long_causal", "tiny", "paged_decode",
+                             "small_decode"])
+    ap.add_argument("--decode-graph", action="store_true",
+                    help="run the decode step as a captured CUDA graph (split pass + merge)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -174,6 +174,37 @@ int paged_attn_decode_noalloc(const attn_bf16* q, const attn_bf16* k_pool, const
                               int max_pages, int num_pages, float scale, void* stream);
 
 /*
+ * Decode as a CUDA graph -- the split pass and the merge of paged_attn_decode
+ * captured once and replayed, which removes the per-call host work and launch
+ * gaps that dominate small-batch decode ("Fast Attention Kernels and Operator
+ * Fusion", section "Fusion and CUDA Graphs with torch.compile": a captured
+ * graph is replayed with one submission; anylearn.cc: capture the decode step
+ * once and replay it, removing per-launch cost).
+ *
+ * paged_attn_decode_graph_create takes exactly the arguments of
+ * paged_attn_decode (minus the stream) and returns an opaque handle in *graph.
+ * The graph keeps every pointer and size it was created with: between
+ * launches the caller may change the CONTENTS of q, k_pool, v_pool,
+ * block_table and seq_lens (same shapes; seq_lens within 1..max_pages *
+ * page_size), and must keep all buffers, the workspace included, alive until
+ * the handle is destroyed.  Creation synchronises nothing but does allocate
+ * host and device resources for the graph; it fails with the status
+ * paged_attn_decode would return for bad arguments.
+ * paged_attn_decode_graph_launch enqueues one decode step on `stream`.
+ * paged_attn_decode_graph_destroy frees the handle (NULL is allowed); the
+ * caller must make sure no launch of it is still running.
+ */
+typedef struct attn_decode_graph attn_decode_graph;
+
+int paged_attn_decode_graph_create(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                                   const int32_t* block_table, const int32_t* seq_lens, int page_size,
+                                   attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
+                                   int max_pages, int num_pages, float scale, void* workspace,
+                                   size_t workspace_bytes, attn_decode_graph** graph);
+int paged_attn_decode_graph_launch(attn_decode_graph* graph, void* stream);
+int paged_attn_decode_graph_destroy(attn_decode_graph* graph);
+
+/*
  * attn_device_status -- synchronises `stream`, then reads and clears the
  * device error word of the current device.  Returns ATTN_OK if no kernel
  * recorded an error since the last call, ATTN_ERR_DEVICE otherwise (the raw

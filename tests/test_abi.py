@@ -97,3 +97,23 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="missing"):
         api.lib()
+
+
+def test_decode_graph_rejects_bad_arguments_on_the_host(lib):
+    import ctypes
+    h = ctypes.c_void_p(123)
+    args = [FAKE] * 5 + [16, FAKE, FAKE, 2, 8, 2, 128, 4, 8, 0.1, FAKE,
+                         lib.paged_attn_decode_workspace_bytes(2, 8, 128, 4, 16)]
+    assert lib.paged_attn_decode_graph_create(*args, None) == 1          # no handle slot
+    bad = list(args)
+    bad[11] = 96                                                          # d
+    assert lib.paged_attn_decode_graph_create(*bad, ctypes.byref(h)) == 2
+    assert h.value is None                                                # cleared on failure
+    bad = list(args)
+    bad[0] = None
+    assert lib.paged_attn_decode_graph_create(*bad, ctypes.byref(h)) == 1
+    bad = list(args)
+    bad[-1] = 8                                                           # workspace too small
+    assert lib.paged_attn_decode_graph_create(*bad, ctypes.byref(h)) == 4
+    assert lib.paged_attn_decode_graph_launch(None, None) == 1
+    assert lib.paged_attn_decode_graph_destroy(None) == 0

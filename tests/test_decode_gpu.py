@@ -153,3 +153,36 @@ def test_invalid_table_entry_is_reported_not_faulted():
                                    inp["scale"])
     assert api.device_status() & (1 << 11)
     assert torch.all(o[1] == 0) and torch.all(torch.isinf(lse[1]))
+
+
+def test_decode_graph_replays_and_follows_in_place_updates():
+    """The captured split + merge gives the eager result, and picks up new
+    contents written into the same buffers between launches."""
+    cfg = W.DecodeConfig("t", 6, 16, 4, 128, 16, 1, 900, seed=31)
+    a = to_cuda(W.make_decode_inputs(cfg, poison_tail=True, seq_lens=[900, 1, 17, 256, 511, 64]))
+    graph = api.DecodeGraph(a["q"], a["k_pool"], a["v_pool"], a["block_table"], a["seq_lens"], a["scale"])
+    try:
+        go, gl = graph.launch()
+        eo, el = api.paged_attn_decode(a["q"], a["k_pool"], a["v_pool"], a["block_table"], a["seq_lens"],
+                                       a["scale"])
+        torch.cuda.synchronize()
+        assert torch.equal(go, eo) and torch.equal(gl, el)
+        # new step: new query, shorter/longer lengths, permuted pages -- same buffers
+        b = W.make_decode_inputs(W.DecodeConfig("t", 6, 16, 4, 128, 16, 1, 900, seed=32),
+                                 seq_lens=[3, 880, 100, 17, 16, 700])
+        nb = b["block_table"].shape[1]
+        a["q"].copy_(b["q"].cuda())
+        a["seq_lens"].copy_(b["seq_lens"].cuda())
+        a["block_table"].fill_(-1)
+        a["block_table"][:, :nb].copy_(b["block_table"].cuda()[:, :a["block_table"].shape[1]])
+        npg = b["num_pages"]
+        a["k_pool"][:npg].copy_(b["k_pool"].cuda())
+        a["v_pool"][:npg].copy_(b["v_pool"].cuda())
+        go, gl = graph.launch()
+        torch.cuda.synchronize()
+        assert api.device_status() == 0
+        host = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in a.items()}
+        ro, rl = oracle_decode(host)
+        assert_close(go.cpu(), gl.cpu(), ro, rl)
+    finally:
+        graph.close()
