@@ -77,21 +77,25 @@ def gqa_kv_head(h_q: int, Hq: int, Hkv: int) -> int:
 
 
 def attention_scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
-                     row_offset: int = 0) -> np.ndarray:
+                     row_offset: int = 0, window_left: int | None = None) -> np.ndarray:
     """S = scale * q k^T + M for one head.
 
     ``q`` holds query rows ``row_offset .. row_offset + len(q) - 1`` of the head;
     ``k`` holds all keys.  With ``causal`` the additive mask M is -inf where the
     key index exceeds the query index ("FlashAttention-Style Kernels",
-    equation with M and the ``is_causal=True`` example).
+    equation with M and the ``is_causal=True`` example).  ``window_left`` = W
+    (a sliding window, one more mask M of that equation) also sets M to -inf
+    where the key index is below query index - W.
     """
     q = _f64(q)
     k = _f64(k)
     s = float(scale) * (q @ k.T)
+    rows = np.arange(row_offset, row_offset + q.shape[0])[:, None]
+    cols = np.arange(k.shape[0])[None, :]
     if causal:
-        rows = np.arange(row_offset, row_offset + q.shape[0])[:, None]
-        cols = np.arange(k.shape[0])[None, :]
         s = np.where(cols > rows, -np.inf, s)
+    if window_left is not None and window_left >= 0:
+        s = np.where(cols < rows - int(window_left), -np.inf, s)
     return s
 
 
@@ -110,15 +114,16 @@ def softmax_with_lse(s: np.ndarray):
 
 
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
-                   causal: bool, row_offset: int = 0):
+                   causal: bool, row_offset: int = 0, window_left: int | None = None):
     """O and LSE for one head: materialise S, then P, then O = P V."""
-    s = attention_scores(q, k, scale, causal, row_offset)
+    s = attention_scores(q, k, scale, causal, row_offset, window_left)
     p, lse = softmax_with_lse(s)
     o = p @ _f64(v)
     return o, lse
 
 
-def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None = None):
+def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None = None,
+                      window_left: int | None = None):
     """Full attention forward for [B, Hq, N, d] queries and [B, Hkv, N, d] K/V.
 
     Returns (O [B, Hq, N, d] float64, LSE [B, Hq, N] float64).  ``row_chunk``
@@ -139,11 +144,13 @@ def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None
             for r0 in range(0, N, step):
                 r1 = min(N, r0 + step)
                 o[b, h, r0:r1], lse[b, h, r0:r1] = attention_head(
-                    q[b, h, r0:r1], k[b, hk], v[b, hk], scale, causal, row_offset=r0)
+                    q[b, h, r0:r1], k[b, hk], v[b, hk], scale, causal, row_offset=r0,
+                    window_left=window_left)
     return o, lse
 
 
-def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
+def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows,
+                   window_left: int | None = None):
     """O and LSE of selected query rows of head (b, h), each row exact.
 
     Used for sampled parity checks at sizes where the full oracle is too slow.
@@ -157,7 +164,7 @@ def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows):
     out_l = np.empty(rows.size, dtype=np.float64)
     for i, r in enumerate(rows):
         qr = _f64(q[b, h, r:r + 1])
-        o_r, l_r = attention_head(qr, kk, vv, scale, causal, row_offset=int(r))
+        o_r, l_r = attention_head(qr, kk, vv, scale, causal, row_offset=int(r), window_left=window_left)
         out_o[i] = o_r[0]
         out_l[i] = l_r[0]
     return out_o, out_l

@@ -255,6 +255,56 @@ def pin_printed_sizes(o):
     assert list(out.shape) == small and list(lse.shape) == small[:3]
 
 
+def pin_window_closed_form(o):
+    """Sliding window W with K == 0: query i sees keys max(0, i-W) .. i (or
+    .. N-1 without the causal mask), all with score 0, so O_i is their mean
+    and LSE_i = log(count)."""
+    rng = _rng(20)
+    N, d = 40, 8
+    q = _rand(rng, 1, 2, N, d)
+    k = np.zeros((1, 2, N, d))
+    v = _rand(rng, 1, 2, N, d)
+    for W in (0, 1, 5, 39):
+        for causal in (True, False):
+            out, lse = o.attention_forward(q, k, v, causal, 0.2, window_left=W)
+            for i in range(N):
+                lo, hi = max(0, i - W), (i if causal else N - 1)
+                assert np.max(np.abs(out[0, :, i] - v[0, :, lo:hi + 1].mean(axis=1))) < 1e-12
+                assert np.max(np.abs(lse[0, :, i] - math.log(hi - lo + 1))) < 1e-12
+
+
+def pin_window_sdpa(o):
+    """Sliding window against PyTorch's fp64 SDPA with an explicit boolean
+    mask, and against the scalar brute force on tiny inputs."""
+    rng = _rng(21)
+    B, Hq, Hkv, N, d = 1, 4, 2, 45, 8
+    q = _rand(rng, B, Hq, N, d)
+    k = _rand(rng, B, Hkv, N, d)
+    v = _rand(rng, B, Hkv, N, d)
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    for W, causal in ((7, True), (0, True), (20, False)):
+        out, lse = o.attention_forward(q, k, v, causal, 0.3, window_left=W)
+        allowed = (j >= i - W) & ((j <= i) if causal else torch.ones_like(j, dtype=torch.bool))
+        tq = torch.from_numpy(q)
+        tk = torch.from_numpy(k).repeat_interleave(Hq // Hkv, dim=1)
+        tv = torch.from_numpy(v).repeat_interleave(Hq // Hkv, dim=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=allowed, scale=0.3)
+        ref_lse = torch.logsumexp((0.3 * (tq @ tk.transpose(-1, -2))).masked_fill(~allowed, float("-inf")), -1)
+        assert np.max(np.abs(out - ref.numpy())) < 1e-12
+        assert np.max(np.abs(lse - ref_lse.numpy())) < 1e-12
+    # scalar brute force: keys outside the window simply do not take part
+    out, lse = o.attention_forward(q[:, :1, :6], k[:, :1, :6], v[:, :1, :6], True, 0.5, window_left=2)
+    for r in range(6):
+        ws = [(j, math.exp(0.5 * math.fsum(float(q[0, 0, r, t]) * float(k[0, 0, j, t]) for t in range(d))))
+              for j in range(max(0, r - 2), r + 1)]
+        z = math.fsum(w for _, w in ws)
+        assert abs(lse[0, 0, r] - math.log(z)) < 1e-12
+        for t in range(d):
+            want = math.fsum(w * float(v[0, 0, j, t]) for j, w in ws) / z
+            assert abs(out[0, 0, r, t] - want) < 1e-12
+
+
 ALL_PINS = [
     pin_rows_sum_to_one,
     pin_constant_v,
@@ -266,4 +316,6 @@ ALL_PINS = [
     pin_block_table_example,
     pin_paged_equals_contiguous,
     pin_printed_sizes,
+    pin_window_closed_form,
+    pin_window_sdpa,
 ]

@@ -77,11 +77,12 @@ def _fresh_oracle():
 
 def _mut_drop_scale(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0: orig(q, k, 1.0, causal, row_offset)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
+        q, k, 1.0, causal, row_offset, window_left)
 
 
 def _mut_mask_includes_diagonal(m):
-    def scores(q, k, scale, causal, row_offset=0):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None):
         s = float(scale) * (np.asarray(q, float) @ np.asarray(k, float).T)
         if causal:
             rows = np.arange(row_offset, row_offset + s.shape[0])[:, None]
@@ -92,7 +93,7 @@ def _mut_mask_includes_diagonal(m):
 
 
 def _mut_mask_off_by_one_late(m):
-    def scores(q, k, scale, causal, row_offset=0):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None):
         s = float(scale) * (np.asarray(q, float) @ np.asarray(k, float).T)
         if causal:
             rows = np.arange(row_offset, row_offset + s.shape[0])[:, None]
@@ -104,11 +105,12 @@ def _mut_mask_off_by_one_late(m):
 
 def _mut_no_mask(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0: orig(q, k, scale, False, row_offset)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
+        q, k, scale, False, row_offset, window_left)
 
 
 def _mut_transposed_scores(m):
-    def scores(q, k, scale, causal, row_offset=0):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None):
         q = np.asarray(q, float)
         k = np.asarray(k, float)
         s = float(scale) * (k @ q.T)
@@ -146,8 +148,8 @@ def _mut_softmax_wrong_axis(m):
 
 
 def _mut_pv_transposed(m):
-    def head(q, k, v, scale, causal, row_offset=0):
-        s = m.attention_scores(q, k, scale, causal, row_offset)
+    def head(q, k, v, scale, causal, row_offset=0, window_left=None):
+        s = m.attention_scores(q, k, scale, causal, row_offset, window_left)
         p, lse = m.softmax_with_lse(s)
         v = np.asarray(v, float)
         if p.shape[0] == p.shape[1]:
@@ -174,7 +176,22 @@ def _mut_page_no_table(m):
 
 def _mut_scale_squared(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0: orig(q, k, scale * scale, causal, row_offset)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
+        q, k, scale * scale, causal, row_offset, window_left)
+
+
+def _mut_window_off_by_one(m):
+    orig = m.attention_scores
+    def scores(q, k, scale, causal, row_offset=0, window_left=None):
+        w = None if window_left is None or window_left < 0 else window_left + 1
+        return orig(q, k, scale, causal, row_offset, w)
+    m.attention_scores = scores
+
+
+def _mut_window_ignored(m):
+    orig = m.attention_scores
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
+        q, k, scale, causal, row_offset, None)
 
 
 MUTANTS = [
@@ -190,6 +207,8 @@ MUTANTS = [
     _mut_pv_transposed,
     _mut_page_slot_swapped,
     _mut_page_no_table,
+    _mut_window_off_by_one,
+    _mut_window_ignored,
 ]
 
 
