@@ -39,6 +39,8 @@ SIGNATURES = {
     "attn_status_string": (ctypes.c_char_p, [_c_i]),
     "attn_last_cuda_error": (_c_i, []),
     "attn_fwd": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p]),
+    "attn_fwd_window": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f,
+                               _c_p]),
     "paged_attn_decode_split_tokens": (_c_i, [_c_i, _c_i, _c_i, _c_i]),
     "paged_attn_decode_workspace_bytes": (_c_sz, [_c_i, _c_i, _c_i, _c_i, _c_i]),
     "paged_attn_decode": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i,
@@ -123,9 +125,10 @@ def _require(t: torch.Tensor, name: str, dtype, ndim: int):
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
              scale: float | None = None, out: torch.Tensor | None = None,
-             lse: torch.Tensor | None = None, stream=None):
+             lse: torch.Tensor | None = None, stream=None, window_left: int | None = None):
     """Fused attention forward.  q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 CUDA.
 
+    ``window_left`` = W restricts query i to keys j >= i - W (sliding window).
     Returns (o [B,Hq,N,d] bf16, lse [B,Hq,N] fp32).
     """
     _require(q, "q", torch.bfloat16, 4)
@@ -143,9 +146,15 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = T
         lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     _require(out, "out", torch.bfloat16, 4)
     _require(lse, "lse", torch.float32, 3)
-    rc = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                        B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
-    _check(rc, "attn_fwd")
+    if window_left is None:
+        rc = lib().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                            B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
+        _check(rc, "attn_fwd")
+    else:
+        rc = lib().attn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                   B, Hq, Hkv, N, d, int(bool(causal)), int(window_left), float(scale),
+                                   _stream_handle(stream))
+        _check(rc, "attn_fwd_window")
     return out, lse
 
 

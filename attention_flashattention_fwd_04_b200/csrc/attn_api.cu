@@ -92,12 +92,12 @@ int sm_count() {
   return counts[dev];
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool WINDOW>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const attn::PrefillParams& p, cudaStream_t stream) {
   using L = attn::PrefillLayout<D>;
-  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL>;
-  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL>>(L::kAlloc);
+  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, WINDOW>;
+  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL, WINDOW>>(L::kAlloc);
   if (e != cudaSuccess) return fail_cuda(e);
   const int sms = sm_count();
   if (sms <= 0) return fail_cuda(cudaErrorInvalidDevice);
@@ -212,13 +212,15 @@ const char* attn_status_string(int status) {
 
 int attn_last_cuda_error(void) { return t_last_cuda_error; }
 
-int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
-             int B, int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+int attn_fwd_window(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
+                    int B, int Hq, int Hkv, int N, int d, int causal, int window_left, float scale,
+                    void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_SHAPE;
   if (d != 64 && d != 128) return ATTN_ERR_SHAPE;
   if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
   if (causal != 0 && causal != 1) return ATTN_ERR_SHAPE;
+  if (window_left < -1) return ATTN_ERR_SHAPE;
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_SHAPE;
   const long long bh = static_cast<long long>(B) * Hq;
   const long long blocks = (static_cast<long long>(N) + 255) / 256;
@@ -245,11 +247,23 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
   p.group = Hq / Hkv;
   p.num_m = static_cast<int>(blocks);
   p.num_items = static_cast<int>(blocks * bh);
+  p.window_left = window_left >= N - 1 ? -1 : window_left;  // a window covering every key is no window
   p.scale_log2 = scale * kLog2e;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return causal ? launch_prefill<128, true>(tq, tk, tv, p, s) : launch_prefill<128, false>(tq, tk, tv, p, s);
-  return causal ? launch_prefill<64, true>(tq, tk, tv, p, s) : launch_prefill<64, false>(tq, tk, tv, p, s);
+  const bool win = p.window_left >= 0;
+  if (d == 128) {
+    if (win)
+      return causal ? launch_prefill<128, true, true>(tq, tk, tv, p, s) : launch_prefill<128, false, true>(tq, tk, tv, p, s);
+    return causal ? launch_prefill<128, true, false>(tq, tk, tv, p, s) : launch_prefill<128, false, false>(tq, tk, tv, p, s);
+  }
+  if (win)
+    return causal ? launch_prefill<64, true, true>(tq, tk, tv, p, s) : launch_prefill<64, false, true>(tq, tk, tv, p, s);
+  return causal ? launch_prefill<64, true, false>(tq, tk, tv, p, s) : launch_prefill<64, false, false>(tq, tk, tv, p, s);
+}
+
+int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B,
+             int Hq, int Hkv, int N, int d, int causal, float scale, void* stream) {
+  return attn_fwd_window(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, -1, scale, stream);
 }
 
 int paged_attn_decode_split_tokens(int num_seqs, int Hkv, int max_pages, int page_size) {

@@ -66,6 +66,7 @@ struct PrefillParams {
   int group;         // Hq / Hkv
   int num_m;         // ceil(N / 256): 256-row query blocks per head
   int num_items;     // B * Hq * num_m
+  int window_left;   // query i sees keys >= i - window_left (kernels with WINDOW only)
   float scale_log2;  // scale * log2(e)
 };
 
@@ -106,14 +107,20 @@ struct PrefillLayout {
   static constexpr uint32_t kColO = 256;        // O0 at 256, O1 at 256 + D
 };
 
-// One work item: 256 query rows [m*256, m*256+256) of head (b, h).
+// One work item: 256 query rows [m*256, m*256+256) of head (b, h).  Query
+// tile t (rows m*256 + 128t ...) sees the 128-key KV tiles j with
+// lo[t] <= j < hi[t]; the item walks j over [jb, je), the union of both.
 struct PrefillItem {
   int b, h, m;
-  int n0, n1;   // KV tiles seen by Q0 / Q1 (n1 = 0 when Q1 lies past N)
-  int n_kv;     // max(n0, n1)
+  int lo0, hi0, lo1, hi1;  // tile 1 is empty (lo1 = hi1) when its rows lie past N
+  int jb, je;
+  __device__ __forceinline__ int lo(int t) const { return t ? lo1 : lo0; }
+  __device__ __forceinline__ int hi(int t) const { return t ? hi1 : hi0; }
+  __device__ __forceinline__ bool active(int t, int j) const { return lo(t) <= j && j < hi(t); }
+  __device__ __forceinline__ bool has(int t) const { return hi(t) > lo(t); }
 };
 
-template <bool CAUSAL>
+template <bool CAUSAL, bool WINDOW>
 __device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, PrefillItem& it) {
   const int G = static_cast<int>(gridDim.x);
   const int c = static_cast<int>(blockIdx.x);
@@ -125,16 +132,28 @@ __device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, 
   const int bh = idx % bh_count;
   it.b = bh / p.Hq;
   it.h = bh % p.Hq;
-  const int n_all = (p.N + 127) / 128;
-  const bool has_q1 = it.m * 256 + 128 < p.N;
-  if (CAUSAL) {
-    it.n0 = min(2 * it.m + 1, n_all);
-    it.n1 = has_q1 ? min(2 * it.m + 2, n_all) : 0;
-  } else {
-    it.n0 = n_all;
-    it.n1 = has_q1 ? n_all : 0;
+  // Tile t: rows r0 .. r0+127; visible keys from first (window) to last
+  // (causal diagonal or N - 1).
+  {
+    const int r0 = it.m * 256;
+    const int first_key = WINDOW ? max(0, r0 - p.window_left) : 0;
+    const int last_key = CAUSAL ? min(r0 + 127, p.N - 1) : p.N - 1;
+    it.lo0 = first_key / 128;
+    it.hi0 = last_key / 128 + 1;
   }
-  it.n_kv = max(it.n0, it.n1);
+  {
+    const int r0 = it.m * 256 + 128;
+    if (r0 >= p.N) {
+      it.lo1 = it.hi1 = 0;
+    } else {
+      const int first_key = WINDOW ? max(0, r0 - p.window_left) : 0;
+      const int last_key = CAUSAL ? min(r0 + 127, p.N - 1) : p.N - 1;
+      it.lo1 = first_key / 128;
+      it.hi1 = last_key / 128 + 1;
+    }
+  }
+  it.jb = it.lo0;
+  it.je = max(it.hi0, it.has(1) ? it.hi1 : 0);
   return true;
 }
 
@@ -150,7 +169,7 @@ __device__ __forceinline__ void reg_alloc_control() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool WINDOW>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -234,24 +253,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ++v_issued;
         return true;
       };
-      for (int r = 0; ok && prefill_item<CAUSAL>(r, p, it); ++r) {
+      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
         const int qz = it.b * p.Hq + it.h;
         const int kz = it.b * p.Hkv + it.h / p.group;  // GQA: consecutive query heads share a KV head
-        // K_0 first: it can land while the previous item still holds Q.
-        if (!(ok = load_k(0, kz))) break;
+        // The item's first K tile first: it can land while the previous item
+        // still holds Q.
+        if (!(ok = load_k(it.jb, kz))) break;
         if (r > 0 && !(ok = mbar_wait(bar(L::kBarQEmpty), static_cast<uint32_t>(r - 1) & 1u, kErrWaitQ)))
           break;
-        mbar_arrive_expect_tx(bar(L::kBarQFull), (it.n1 > 0 ? 2 : 1) * L::kTileBytes);
+        mbar_arrive_expect_tx(bar(L::kBarQFull), (it.has(1) ? 2 : 1) * L::kTileBytes);
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(base + L::kQ0 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, it.m * 256, qz);
-        if (it.n1 > 0)
+        if (it.has(1))
           for (int c = 0; c < D / 64; ++c)
             tma_load_3d(base + L::kQ1 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, it.m * 256 + 128,
                         qz);
         ++q_issued;
-        if (!(ok = load_v(0, kz))) break;
+        if (!(ok = load_v(it.jb, kz))) break;
         ++kv_it;
-        for (int j = 1; j < it.n_kv; ++j, ++kv_it) {
+        for (int j = it.jb + 1; j < it.je; ++j, ++kv_it) {
           if (!(ok = load_k(j, kz))) break;
           if (!(ok = load_v(j, kz))) break;
         }
@@ -293,69 +313,71 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                       idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
       };
       PrefillItem it;
-      for (int r = 0; ok && prefill_item<CAUSAL>(r, p, it); ++r) {
+      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
         if (!(ok = mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(r) & 1u, kErrWaitQ))) break;
+        const int nkv = it.je - it.jb;
         {
           const int st = kv_it % NS;
           if (!(ok = mbar_wait(bar(L::kBarKFull + st), static_cast<uint32_t>(kv_it / NS) & 1u, kErrWaitKFull)))
             break;
           tc_fence_after();
-          issue_s(0, st);
-          if (it.n1 > 0) issue_s(1, st);
+          if (it.active(0, it.jb)) issue_s(0, st);
+          if (it.active(1, it.jb)) issue_s(1, st);
           mma_commit(bar(L::kBarKEmpty + st));
-          if (it.n_kv == 1) mma_commit(bar(L::kBarQEmpty));  // last S of the item: Q may be replaced
+          if (nkv == 1) mma_commit(bar(L::kBarQEmpty));  // last S of the item: Q may be replaced
         }
-        for (int j = 0; j < it.n_kv && ok; ++j) {
-          const int g = kv_it + j;
+        for (int j = it.jb; j < it.je && ok; ++j) {
+          const int g = kv_it + (j - it.jb);
           const int st = g % NS, st1 = (g + 1) % NS;
           const uint32_t ph = static_cast<uint32_t>(g / NS) & 1u, ph1 = static_cast<uint32_t>((g + 1) / NS) & 1u;
           bool v_ready = false, k_ready = false;
-          if (j < it.n0) {
+          if (it.active(0, j)) {
             const uint32_t pph = p_cnt[0]++ & 1u;
             if (!(ok = mbar_wait(bar(L::kBarPFull + 0), pph, kErrWaitPFull))) break;
-            if (j == 0 && o_cnt[0] > 0 &&
+            if (j == it.lo0 && o_cnt[0] > 0 &&
                 !(ok = mbar_wait(bar(L::kBarOFree + 0), (o_cnt[0] - 1u) & 1u, kErrWaitODone)))
               break;
             if (!(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
             v_ready = true;
             tc_fence_after();
-            issue_pv(0, st, j > 0);
-            if (j + 1 == it.n0) {
+            issue_pv(0, st, j > it.lo0);
+            if (j + 1 == it.hi0) {
               mma_commit(bar(L::kBarOFull + 0));  // O0 of this item is final once this lands
               ++o_cnt[0];
             }
-            if (j + 1 < it.n0) {
+            if (it.active(0, j + 1)) {
               if (!(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
               k_ready = true;
               tc_fence_after();
               issue_s(0, st1);
             }
           }
-          if (j < it.n1) {
+          if (it.active(1, j)) {
             const uint32_t pph = p_cnt[1]++ & 1u;
             if (!(ok = mbar_wait(bar(L::kBarPFull + 1), pph, kErrWaitPFull))) break;
-            if (j == 0 && o_cnt[1] > 0 &&
+            if (j == it.lo1 && o_cnt[1] > 0 &&
                 !(ok = mbar_wait(bar(L::kBarOFree + 1), (o_cnt[1] - 1u) & 1u, kErrWaitODone)))
               break;
             if (!v_ready && !(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
             tc_fence_after();
-            issue_pv(1, st, j > 0);
-            if (j + 1 == it.n1) {
+            issue_pv(1, st, j > it.lo1);
+            if (j + 1 == it.hi1) {
               mma_commit(bar(L::kBarOFull + 1));
               ++o_cnt[1];
             }
-            if (j + 1 < it.n1) {
-              if (!k_ready && !(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
-              tc_fence_after();
-              issue_s(1, st1);
-            }
+          }
+          if (it.active(1, j + 1)) {
+            // Q1's next S; also its first one when its window starts at j + 1.
+            if (!k_ready && !(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
+            tc_fence_after();
+            issue_s(1, st1);
           }
           mma_commit(bar(L::kBarVEmpty + st));
-          if (j + 1 < it.n_kv) mma_commit(bar(L::kBarKEmpty + st1));
-          if (j + 2 == it.n_kv) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
+          if (j + 1 < it.je) mma_commit(bar(L::kBarKEmpty + st1));
+          if (j + 2 == it.je) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
         }
         if (!ok) break;
-        kv_it += it.n_kv;
+        kv_it += nkv;
       }
       // All issued MMAs must finish before tensor memory is released.
       mma_commit(bar(L::kBarMmaDone));
@@ -370,10 +392,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t st_cnt[2] = {0u, 0u};  // items whose tile t this warpgroup has written out
     bool ok = true;
     PrefillItem it;
-    for (int r = 0; ok && prefill_item<CAUSAL>(r, p, it); ++r) {
+    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if ((t == 0 ? it.n0 : it.n1) == 0) continue;
+        if (!it.has(t)) continue;
         const uint32_t n = st_cnt[t];
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarOFull + t), n & 1u, kErrWaitODone));
         if (!ok) break;
@@ -424,14 +446,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t s_cnt = 0, st_cnt = 0;
     bool ok = true;
     PrefillItem it;
-    for (int r = 0; ok && prefill_item<CAUSAL>(r, p, it); ++r) {
-      const int n_t = t ? it.n1 : it.n0;
+    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
+      const int lo_t = it.lo(t);
+      const int n_t = it.hi(t) - lo_t;  // KV tiles this query tile visits (>= 0)
       if (n_t == 0) continue;
-      const int grow = it.m * 256 + t * 128 + row;
-      const int diag = 2 * it.m + t;  // KV tile holding this query tile's diagonal
-      float m_used = -INFINITY;       // running max in scaled log2 units
+      const int row0 = it.m * 256 + t * 128;  // first row of this query tile
+      const int grow = row0 + row;
+      float m_used = -INFINITY;  // running max in scaled log2 units
       float l_sum = 0.f;
-      for (int j = 0; j < n_t; ++j) {
+      for (int jj = 0; jj < n_t; ++jj) {
+        const int j = lo_t + jj;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarSFull + t), s_cnt++ & 1u, kErrWaitSFull));
         if (!ok) break;
         tc_fence_after();
@@ -441,11 +465,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
         const int kv0 = j * 128;
-        if ((CAUSAL && j == diag) || kv0 + 128 > p.N) {
-          const int last = CAUSAL ? min(grow, p.N - 1) : p.N - 1;  // last visible key
+        // Tiles crossing the causal diagonal, a window's left edge or N get a
+        // per-element mask (a select, so NaN-free -inf).
+        if ((CAUSAL && kv0 + 127 > row0) || kv0 + 128 > p.N ||
+            (WINDOW && kv0 < min(row0 + 127, p.N - 1) - p.window_left)) {
+          // Visible keys of this row: [first, last], as offsets into the tile.
+          const int last = (CAUSAL ? min(grow, p.N - 1) : p.N - 1) - kv0;
+          if constexpr (WINDOW) {
+            const int first = grow - p.window_left - kv0;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (kv0 + c > last) s[c] = -INFINITY;
+            for (int c = 0; c < 128; ++c)
+              if (c > last || c < first) s[c] = -INFINITY;
+          } else {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (c > last) s[c] = -INFINITY;
+          }
         }
         // Row max: four chains of three-input maxima.
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
@@ -489,7 +524,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             pk[i] = pack_bf16x2(p0, p1);
           }
           tmem_st_x32(s_addr + static_cast<uint32_t>(half * 32), pk);
-          if (half == 0 && j > 0 && __any_sync(0xffffffffu, upd)) {
+          if (half == 0 && jj > 0 && __any_sync(0xffffffffu, upd)) {
             // O_t is idle here (its last update was issued before S_t of this
             // tile, and this tile's update waits for the barrier below).
 #pragma unroll

@@ -16,6 +16,9 @@ rounded to nearest-even; draw order Q, K, V, then any per-position offset):
 * ``long_causal``  B=1, H=8, N=32768, d=128, causal, N(0,1) with one offset
   c_j ~ N(0, sigma=2) per key position added to every element of key row j
   (shared by all heads) to make peaked softmax rows, seed 5
+* ``long_window``  the ``long_causal`` shapes and draws (seed 7) with a sliding
+  window: query i sees keys i-4095 .. i (a 4096-key window, the size used by
+  common sliding-window models; the pages name the pattern, not a size)
 
 The page size of 16 tokens is the cache block size of the vLLM example in
 "Fast Attention Kernels and Operator Fusion" (wpnews.pro), section "Paged
@@ -38,6 +41,7 @@ __all__ = [
     "make_prefill_inputs",
     "make_decode_inputs",
     "prefill_flops",
+    "visible_pairs",
     "decode_kv_bytes",
 ]
 
@@ -54,6 +58,7 @@ class PrefillConfig:
     seed: int
     value_scale: float = 1.0
     k_offset_sigma: float = 0.0
+    window_left: int = -1  # W >= 0: query i sees keys j >= i - W only; -1: no window
 
     @property
     def scale(self) -> float:
@@ -89,6 +94,8 @@ PREFILL_CONFIGS = {
     "causal_mha": PrefillConfig("causal_mha", 4, 16, 16, 2048, 128, True, 2),
     "causal_gqa": PrefillConfig("causal_gqa", 1, 32, 8, 8192, 128, True, 3, value_scale=0.5),
     "long_causal": PrefillConfig("long_causal", 1, 8, 8, 32768, 128, True, 5, k_offset_sigma=2.0),
+    "long_window": PrefillConfig("long_window", 1, 8, 8, 32768, 128, True, 7, k_offset_sigma=2.0,
+                                 window_left=4095),
 }
 
 DECODE_CONFIGS = {
@@ -171,8 +178,22 @@ def make_decode_inputs(cfg: DecodeConfig, device: str | torch.device = "cpu",
     }
 
 
+def visible_pairs(N: int, causal: bool, window_left: int = -1) -> int:
+    """Number of (query, key) pairs the mask leaves visible in one head."""
+    i = torch.arange(N, dtype=torch.int64)
+    last = i if causal else torch.full_like(i, N - 1)
+    first = (i - window_left).clamp(min=0) if window_left >= 0 else torch.zeros_like(i)
+    return int((last - first + 1).clamp(min=0).sum().item())
+
+
 def prefill_flops(cfg: PrefillConfig) -> float:
-    """Algorithmic FLOPs: 4*B*Hq*N^2*d, halved for causal (QK^T and PV)."""
+    """Algorithmic FLOPs of QK^T and PV: 4*d per visible (query, key) pair.
+
+    Without a window the usual convention is kept: 4*B*Hq*N^2*d, halved for
+    causal.  With a sliding window the visible pairs are counted exactly.
+    """
+    if cfg.window_left >= 0:
+        return 4.0 * cfg.B * cfg.Hq * cfg.d * visible_pairs(cfg.N, cfg.causal, cfg.window_left)
     f = 4.0 * cfg.B * cfg.Hq * cfg.N * cfg.N * cfg.d
     return f / 2.0 if cfg.causal else f
 

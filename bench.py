@@ -13,7 +13,7 @@ i.e. the time-weighted fraction of the measured B200 peaks the step reaches
 separate prefill TFLOP/s and decode GB/s are in the line too.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--workload default|causal_mha|causal_gqa|long_causal|paged_decode|small_decode]
+       [--workload default|causal_mha|causal_gqa|long_causal|long_window|paged_decode|small_decode]
        [--decode-graph]
 Under torchrun each rank runs its own batch (seed offset by rank), no
 collective on the data path; rank 0 prints one JSON line.
@@ -22,6 +22,7 @@ collective on the data path; rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -167,6 +168,16 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
+PREFILL_WORKLOADS = ("default", "causal_mha", "causal_gqa", "long_causal", "long_window", "tiny")
+DECODE_WORKLOADS = ("default", "paged_decode", "small_decode")
+
+
+def prefill_label(c) -> str:
+    mask = "causal" if c.causal else "full"
+    if c.window_left >= 0:
+        mask += f" window={c.window_left}"
+    return f"{mask} prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}"
+
 class Step:
     """Device-resident inputs/outputs for one rank and the calls of one step."""
 
@@ -176,12 +187,11 @@ class Step:
         self.device = device
         self.prefill_cfg = None
         self.decode_cfg = None
-        if workload in ("default", "causal_mha", "causal_gqa", "long_causal", "tiny"):
+        if workload in PREFILL_WORKLOADS:
             name = "causal_mha" if workload == "default" else workload
             base = W.PREFILL_CONFIGS[name]
-            self.prefill_cfg = W.PrefillConfig(base.name, base.B, base.Hq, base.Hkv, base.N, base.d, base.causal,
-                                               shard_seed(base.seed, rank), base.value_scale, base.k_offset_sigma)
-        if workload in ("default", "paged_decode", "small_decode"):
+            self.prefill_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
+        if workload in DECODE_WORKLOADS:
             base = W.DECODE_CONFIGS["small_decode" if workload == "small_decode" else "paged_decode"]
             self.decode_cfg = W.DecodeConfig(base.name, base.num_seqs, base.Hq, base.Hkv, base.d, base.page_size,
                                              base.min_len, base.max_len, shard_seed(base.seed, rank))
@@ -229,7 +239,8 @@ class Step:
     def run_prefill(self, d=None):
         d = d or self.dev
         c = self.prefill_cfg
-        self.api.attn_fwd(d["q"], d["k"], d["v"], c.causal, c.scale, out=d["o"], lse=d["lse"])
+        self.api.attn_fwd(d["q"], d["k"], d["v"], c.causal, c.scale, out=d["o"], lse=d["lse"],
+                          window_left=c.window_left if c.window_left >= 0 else None)
 
     def run_decode(self, d=None):
         d = d or self.dev
@@ -249,10 +260,10 @@ def config_dict(step: Step, n_gpus: int):
     parts = []
     if step.prefill_cfg is not None:
         c = step.prefill_cfg
-        parts.append(f"causal prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}")
+        parts.append(prefill_label(c))
         cfg["prefill"] = {"B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "N": c.N, "d": c.d, "causal": c.causal,
-                          "scale": c.scale, "seed": c.seed, "value_scale": c.value_scale,
-                          "k_offset_sigma": c.k_offset_sigma, "flops": step.flops}
+                          "window_left": c.window_left, "scale": c.scale, "seed": c.seed,
+                          "value_scale": c.value_scale, "k_offset_sigma": c.k_offset_sigma, "flops": step.flops}
     if step.decode_cfg is not None:
         c = step.decode_cfg
         L = step.decode_inp["seq_lens"]
@@ -266,7 +277,7 @@ def config_dict(step: Step, n_gpus: int):
     if step.decode_cfg is not None:
         cfg["l2"] = "inputs larger than L2: the decode pass streams >1 GB of KV through the 126 MB L2 every step"
     else:
-        cfg["l2"] = "L2 flushed between steps (256 MB write)"
+        cfg["l2"] = "L2 flushed between steps (256 MB write, outside the timed regions)"
     return cfg
 
 
@@ -297,10 +308,14 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
             for h in range(c.Hq):
                 hk = h * c.Hkv // c.Hq
                 r0 = c.N - rows
-                oracle.attention_head(q[b, h, r0:], k[b, hk], v[b, hk], c.scale, c.causal, row_offset=r0)
-                # causal work of rows r0..N-1: sum over rows of (row+1) keys
-                keys = (rows * (r0 + 1 + c.N)) / 2.0 if c.causal else rows * c.N
-                flops += 4.0 * keys * c.d
+                wl = c.window_left if c.window_left >= 0 else None
+                oracle.attention_head(q[b, h, r0:], k[b, hk], v[b, hk], c.scale, c.causal, row_offset=r0,
+                                      window_left=wl)
+                # visible (query, key) pairs of rows r0..N-1
+                i = np.arange(r0, c.N)
+                last = i if c.causal else np.full_like(i, c.N - 1)
+                first = np.maximum(i - wl, 0) if wl is not None else np.zeros_like(i)
+                flops += 4.0 * float(np.sum(last - first + 1)) * c.d
                 done_heads += 1
                 if time.perf_counter() - t0 > budget_s / (2 if decode_cfg is not None else 1):
                     break
@@ -381,14 +396,13 @@ class StepHost:
         self.host = {}
         self.decode_inp = None
         parts = []
-        if workload in ("default", "causal_mha", "causal_gqa", "long_causal", "tiny"):
+        if workload in PREFILL_WORKLOADS:
             name = "causal_mha" if workload == "default" else workload
             self.prefill_cfg = W.PREFILL_CONFIGS[name]
             q, k, v = W.make_prefill_inputs(self.prefill_cfg)
             self.host.update(q=q, k=k, v=v)
-            c = self.prefill_cfg
-            parts.append(f"causal prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}")
-        if workload in ("default", "paged_decode", "small_decode"):
+            parts.append(prefill_label(self.prefill_cfg))
+        if workload in DECODE_WORKLOADS:
             self.decode_cfg = W.DECODE_CONFIGS["small_decode" if workload == "small_decode" else "paged_decode"]
             inp = W.make_decode_inputs(self.decode_cfg)
             self.decode_inp = inp
@@ -461,6 +475,10 @@ def run_ours(args, world, rank, local_rank):
         if step.decode_cfg is not None:
             a = evs[i][1] if step.prefill_cfg is not None else (evs[i - 1][2] if i > 0 else start)
             t_decode += a.elapsed_time(evs[i][2]) / 1e3
+    if flush is not None:
+        # The L2 flush between steps is not work of the step: time the steps'
+        # own event-bracketed regions (each one starts with a cold L2).
+        total_s = t_prefill
     t_max = max_over_ranks(total_s, world, device)
     ideal_sum = sum_over_ranks(step.ideal_seconds(peaks) * args.steps, world, device)
     value = ideal_sum / t_max
@@ -567,8 +585,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="default",
-                    choices=["default", "causal_mha", "causal_gqa", "long_causal", "tiny", "paged_decode",
-                             "small_decode"])
+                    choices=sorted(set(PREFILL_WORKLOADS) | set(DECODE_WORKLOADS)))
     ap.add_argument("--decode-graph", action="store_true",
                     help="run the decode step as a captured CUDA graph (split pass + merge)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

@@ -82,6 +82,24 @@ int attn_fwd(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf
              void* stream);
 
 /*
+ * attn_fwd_window -- attn_fwd with a sliding window: query i sees the keys j
+ * with i - window_left <= j (and j <= i when causal), i.e. the additive mask M
+ * of the attention equation is also -inf left of the window.  The pattern is
+ * named beside causal as a standard mask that keeps a fused path in use
+ * ("Finding the Next One: Fusion Beyond Attention", anylearn.cc, on silent
+ * fallbacks) and as the Longformer-style window of block-sparse attention
+ * ("Kernel Fusion and Custom Kernels", ai.zenoagi.com, section 4 on
+ * FlashInfer); no page fixes its size.  window_left = -1
+ * means no left limit (attn_fwd is this call with -1); window_left = 0 with
+ * causal = 1 lets each query see only itself.  KV tiles wholly outside every
+ * row's window are skipped, so the work is O(N * window) instead of O(N^2).
+ * Errors: those of attn_fwd, plus ATTN_ERR_SHAPE for window_left < -1.
+ */
+int attn_fwd_window(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o,
+                    float* lse, int B, int Hq, int Hkv, int N, int d, int causal, int window_left,
+                    float scale, void* stream);
+
+/*
  * paged_attn_decode_split_tokens -- tokens per split of the split-KV decode
  * pass for this problem shape (a multiple of 16).  The split plan depends only
  * on these arguments, never on the sequence lengths, so the host never has to

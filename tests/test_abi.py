@@ -51,6 +51,13 @@ def test_attn_fwd_rejects(lib, kw, code):
     assert _fwd(lib, **kw) == code
 
 
+@pytest.mark.parametrize("wl,code", [(-2, 2), (-100, 2)])
+def test_attn_fwd_window_rejects(lib, wl, code):
+    assert lib.attn_fwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 16, 64, 1, wl, 0.125, None) == code
+    assert lib.attn_fwd_window(None, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 16, 64, 1, 4, 0.125, None) == 1
+    assert lib.attn_fwd_window(FAKE + 8, FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 16, 64, 1, 4, 0.125, None) == 3
+
+
 def _dec(lib, q=FAKE, kp=FAKE, vp=FAKE, bt=FAKE, sl=FAKE, ps=16, o=FAKE, lse=FAKE, S=2, Hq=8, Hkv=2,
          d=128, max_pages=4, num_pages=8, scale=0.1, ws=FAKE, ws_bytes=None):
     if ws_bytes is None:

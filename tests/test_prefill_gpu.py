@@ -24,8 +24,8 @@ def f64(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def run_gpu(q, k, v, causal, scale):
-    o, lse = api.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal, scale)
+def run_gpu(q, k, v, causal, scale, window_left=None):
+    o, lse = api.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal, scale, window_left=window_left)
     assert api.device_status() == 0
     return f64(o), f64(lse)
 
@@ -74,7 +74,8 @@ def test_tiny_config_full():
 
 def _sampled(cfg, heads, rows, seed):
     q, k, v = W.make_prefill_inputs(cfg)
-    o, lse = api.attn_fwd(q.cuda(), k.cuda(), v.cuda(), cfg.causal, cfg.scale)
+    wl = cfg.window_left if cfg.window_left >= 0 else None
+    o, lse = api.attn_fwd(q.cuda(), k.cuda(), v.cuda(), cfg.causal, cfg.scale, window_left=wl)
     assert api.device_status() == 0
     o = o.float().cpu()
     lse = lse.cpu()
@@ -82,7 +83,7 @@ def _sampled(cfg, heads, rows, seed):
     rng = np.random.default_rng(seed)
     for (b, h) in heads:
         rr = sorted(set(rows) | set(rng.integers(0, cfg.N, 12).tolist()))
-        ro, rl = oracle.attention_rows(q, k, v, cfg.causal, cfg.scale, b, h, rr)
+        ro, rl = oracle.attention_rows(q, k, v, cfg.causal, cfg.scale, b, h, rr, window_left=wl)
         got_o = o[b, h, rr].numpy().astype(np.float64)
         got_l = lse[b, h, rr].numpy().astype(np.float64)
         assert_close(got_o, got_l, ro, rl)
@@ -101,6 +102,11 @@ def test_causal_gqa_full_size_sampled():
 def test_long_causal_full_size_sampled():
     cfg = W.PREFILL_CONFIGS["long_causal"]
     _sampled(cfg, [(0, 0), (0, 7)], [0, 1, 128, 16383, 32766, 32767], 5)
+
+
+def test_long_window_full_size_sampled():
+    cfg = W.PREFILL_CONFIGS["long_window"]
+    _sampled(cfg, [(0, 0), (0, 5)], [0, 1, 4095, 4096, 4097, 8191, 8192, 20000, 32767], 7)
 
 
 def test_causal_mha_whole_heads():
@@ -157,3 +163,74 @@ def test_memory_does_not_scale_with_n_squared():
         torch.cuda.synchronize()
         free.append(before - torch.cuda.mem_get_info()[0])
     assert max(free) <= 2 * 1024 * 1024, free
+
+
+# -- sliding window ----------------------------------------------------------------
+
+WINDOW = [
+    # B, Hq, Hkv, N, d, causal, W (query i sees keys i-W .. i, or i-W .. N-1 when not causal)
+    (1, 2, 2, 1, 64, True, 0),
+    (1, 2, 1, 300, 128, True, 0),
+    (1, 2, 2, 300, 128, True, 1),
+    (1, 4, 2, 513, 128, True, 127),
+    (1, 4, 2, 513, 64, True, 128),
+    (2, 2, 2, 700, 128, True, 129),
+    (1, 2, 2, 1000, 128, True, 255),
+    (1, 8, 2, 1300, 128, True, 500),
+    (1, 3, 3, 129, 128, False, 0),
+    (1, 2, 2, 1000, 64, False, 300),
+    (1, 2, 1, 640, 128, False, 129),
+    (1, 2, 2, 777, 128, True, 776),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal,wl", WINDOW)
+def test_sliding_window_small_shapes(B, Hq, Hkv, N, d, causal, wl):
+    cfg = W.PrefillConfig("t", B, Hq, Hkv, N, d, causal, seed=300 + N + wl)
+    q, k, v = W.make_prefill_inputs(cfg)
+    o, lse = run_gpu(q, k, v, causal, cfg.scale, window_left=wl)
+    ro, rl = oracle.attention_forward(f64(q), f64(k), f64(v), causal, cfg.scale, window_left=wl)
+    assert_close(o, lse, ro, rl)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_window_covering_every_key_is_no_window(causal):
+    """W >= N - 1 hides nothing: the result is the unwindowed one, bit for bit."""
+    cfg = W.PrefillConfig("t", 1, 4, 2, 384, 128, causal, seed=41)
+    q, k, v = (t.cuda() for t in W.make_prefill_inputs(cfg))
+    a = api.attn_fwd(q, k, v, causal, cfg.scale)
+    for wl in (383, 10 ** 6):
+        b = api.attn_fwd(q, k, v, causal, cfg.scale, window_left=wl)
+        torch.cuda.synchronize()
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("j0,wl", [(77, 0), (127, 128), (200, 129), (383, 255), (5, 600)])
+def test_window_edges_are_exact(j0, wl, causal):
+    """Key j0 scores ~255 (log2 units) above every other key, so a row that
+    sees it returns V[j0] bit for bit and a row that does not cannot.  Row
+    j0 + W is the last to see it (the left edge is inclusive); row j0 + W + 1
+    is the first that does not; with causal, rows before j0 do not either."""
+    N, d = 1024, 128
+    q = torch.zeros(1, 2, N, d)
+    q[..., 0] = 1.0
+    g = torch.Generator().manual_seed(8)
+    k = torch.randn(1, 2, N, d, generator=g) * 0.01
+    k[..., j0, 0] = 2000.0
+    v = torch.randn(1, 2, N, d, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    o, lse = api.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal, scale, window_left=wl)
+    assert api.device_status() == 0
+    o = o.cpu()
+    first_row = j0 if causal else 0
+    last_row = min(N - 1, j0 + wl)
+    want = v[:, :, j0:j0 + 1, :].expand(1, 2, last_row - first_row + 1, d)
+    assert torch.equal(o[:, :, first_row:last_row + 1], want)
+    outside = [r for r in (first_row - 1, last_row + 1) if 0 <= r < N]
+    for r in outside:
+        assert not torch.equal(o[0, 0, r], v[0, 0, j0])
+    ro, rl = oracle.attention_rows(f64(q), f64(k), f64(v), causal, scale, 0, 1, outside + [last_row],
+                                   window_left=wl)
+    assert_close(f64(o[0, 1, outside + [last_row]]), f64(lse[0, 1, outside + [last_row]]), ro, rl)

@@ -91,3 +91,24 @@ def test_flop_convention():
     assert abs(W.prefill_flops(c2) - 68.72e9) / 68.72e9 < 1e-3
     c3 = W.PREFILL_CONFIGS["causal_gqa"]
     assert abs(W.prefill_flops(c3) - 549.76e9) / 549.76e9 < 1e-3
+
+
+def test_visible_pairs_match_the_oracle_mask():
+    """The windowed FLOP count equals the number of finite scores the oracle's
+    mask leaves, on small shapes (including windows past either end)."""
+    import numpy as np
+    import oracle
+    rng = np.random.default_rng(0)
+    for N in (1, 5, 130, 257):
+        q = rng.standard_normal((N, 4))
+        for causal in (True, False):
+            for wl in (-1, 0, 1, 3, 127, 128, N - 1, N + 5):
+                s = oracle.attention_scores(q, q, 1.0, causal, 0, None if wl < 0 else wl)
+                assert W.visible_pairs(N, causal, wl) == int(np.isfinite(s).sum()), (N, causal, wl)
+
+
+def test_window_flops():
+    lw = W.PREFILL_CONFIGS["long_window"]
+    N, Wl = lw.N, lw.window_left
+    pairs = (Wl + 1) * (Wl + 2) // 2 + (N - Wl - 1) * (Wl + 1)  # ramp, then full windows
+    assert W.prefill_flops(lw) == 4.0 * lw.B * lw.Hq * lw.d * pairs
