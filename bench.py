@@ -41,7 +41,7 @@ from attention_flashattention_fwd_04_b200 import workloads as W  # noqa: E402
 
 METRIC = "causal prefill TFLOP/s and paged-decode KV GB/s, as fraction of B200 peaks"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
-KERNEL_SOURCES = ["attn_api.cu", "prefill_sm100.cuh", "decode_sm100.cuh", "ptx.cuh", "tmem_ldst.cuh"]
+KERNEL_SOURCES = ("attn_api.cu", "prefill_sm100.cuh", "decode_sm100.cuh", "ptx.cuh", "tmem_ldst.cuh", "exp2_poly.cuh")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -79,7 +79,7 @@ def load_traffic():
                     continue
                 kv = dict(tok.split("=", 1) for tok in line.split() if "=" in tok)
                 if "kernel" in kv and "dram_bytes_per_launch" in kv:
-                    out[kv["kernel"]] = (kv.get("sha"), float(kv["dram_bytes_per_launch"]))
+                    out[(kv["kernel"], kv.get("bench"))] = (kv.get("sha"), float(kv["dram_bytes_per_launch"]))
     except OSError:
         return {}
     sha = kernel_source_hash()
@@ -514,9 +514,9 @@ def run_ours(args, world, rank, local_rank):
     traffic = load_traffic()
     dk = kernels[dominant]
     if dominant.startswith("prefill"):
-        tr = traffic.get("prefill_fwd_kernel")
+        tr = traffic.get(("prefill_fwd_kernel", step.prefill_cfg.name))
     else:
-        parts = [traffic.get("decode_split_kernel"), traffic.get("decode_merge_kernel")]
+        parts = [traffic.get((k, step.decode_cfg.name)) for k in ("decode_split_kernel", "decode_merge_kernel")]
         tr = None if any(x is None for x in parts) else sum(parts)
     line["roofline"] = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
                         "unit": dk["unit"], "frac": dk["frac"], "traffic": tr,
