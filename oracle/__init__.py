@@ -11,6 +11,8 @@ from .attention import (  # noqa: F401
     attention_scores,
     gather_paged_kv,
     gqa_kv_head,
+    paged_append,
     paged_decode,
+    paged_prefill,
     softmax_with_lse,
 )

@@ -35,13 +35,27 @@ Readings where the pages are silent (each is restated where it is used):
   t % page_size ("Paged Attention Kernels" section and its block-table figure,
   logical blocks 0,1,2,3 -> physical 17,4,29,8).  Decode has one query per
   sequence that sees all seq_len cached keys.
+* appending to the cache / chunked prefill ("Operator Fusion" section: the
+  KV cache is updated as keys and values are produced; "Paged Attention
+  Kernels": blocks are allocated as the cache grows): a sequence holding
+  seq_len tokens after the step received its last q_len of them in this step,
+  packed by sequence ([total_q, H, d], rows cu_seqlens_q[s] ..
+  cu_seqlens_q[s+1]-1).  New token i is logical token ctx + i with
+  ctx = seq_len - q_len; its K and V are written there, and its query sees
+  keys 0 .. ctx + i under the causal mask (every one of the seq_len keys
+  without it).
 
 Pins (all in ``tests/test_oracle.py``): rows of P sum to one; constant V rows
 are returned unchanged; K == 0 gives the prefix mean of V and LSE = log(count);
 causal row 0 returns v_0 with LSE = scale q_0 . k_0; a pure-Python ``math.fsum``
 brute force on tiny inputs; PyTorch's fp64 CPU ``scaled_dot_product_attention``
 and ``logsumexp`` as a library special case; the pages' block-table example;
-paged gather equal to contiguous KV bit for bit.
+paged gather equal to contiguous KV bit for bit; the sliding window against a
+closed form, a scalar brute force and SDPA with an explicit mask; the append
+against a hand-worked placement on the pages' block table; chunked prefill
+against SDPA with an explicit bottom-right mask, a scalar brute force, the
+whole-sequence prefill (two chunks give the same rows) and the decode (its
+last row).
 """
 
 from __future__ import annotations
@@ -57,6 +71,8 @@ __all__ = [
     "attention_rows",
     "gather_paged_kv",
     "paged_decode",
+    "paged_append",
+    "paged_prefill",
 ]
 
 
@@ -209,4 +225,70 @@ def paged_decode(q, k_pool, v_pool, block_table, seq_lens, page_size: int, scale
             o_h, l_h = attention_head(q[s, h][None, :], ks[:, hk], vs[:, hk], scale, causal=False)
             o[s, h] = o_h[0]
             lse[s, h] = l_h[0]
+    return o, lse
+
+
+def _chunk_bounds(cu_seqlens_q, seq_lens, s):
+    """(first packed row, q_len, ctx) of sequence s."""
+    q0 = int(cu_seqlens_q[s])
+    q_len = int(cu_seqlens_q[s + 1]) - q0
+    ctx = int(seq_lens[s]) - q_len
+    if q_len < 0 or ctx < 0:
+        raise ValueError("a sequence has more new tokens than tokens in all")
+    return q0, q_len, ctx
+
+
+def paged_append(k_pool, v_pool, k_new, v_new, block_table, cu_seqlens_q, seq_lens, page_size: int):
+    """Write each sequence's new K/V rows into the paged cache.
+
+    k_new/v_new: [total_q, Hkv, d], packed by sequence as the queries are.
+    Row i of sequence s becomes logical token ctx + i, stored at physical page
+    block_table[s][(ctx + i) // page_size], slot (ctx + i) % page_size.
+    Returns new pool arrays (the inputs are not modified); every other slot
+    keeps its old contents.  Pure indexing: exact in the pools' own dtype.
+    """
+    kp = np.array(k_pool, copy=True)
+    vp = np.array(v_pool, copy=True)
+    kn = np.asarray(k_new)
+    vn = np.asarray(v_new)
+    table = np.asarray(block_table)
+    for s in range(len(seq_lens)):
+        q0, q_len, ctx = _chunk_bounds(cu_seqlens_q, seq_lens, s)
+        for i in range(q_len):
+            t = ctx + i
+            page = int(table[s, t // page_size])
+            if page < 0 or page >= kp.shape[0]:
+                raise IndexError("block table entry outside the pool")
+            kp[page, t % page_size] = kn[q0 + i]
+            vp[page, t % page_size] = vn[q0 + i]
+    return kp, vp
+
+
+def paged_prefill(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens, page_size: int, scale: float,
+                  causal: bool = True):
+    """Attention of each sequence's new queries over its whole paged cache.
+
+    q: [total_q, Hq, d] packed by sequence; the pools already hold all
+    seq_len tokens of every sequence (the new ones included).  Query i of
+    sequence s is logical token ctx + i, so under the causal mask it is row
+    ctx + i of the sequence's attention (``row_offset`` = ctx).
+    Returns (O [total_q, Hq, d] float64, LSE [total_q, Hq] float64).
+    """
+    q = _f64(q)
+    total_q, Hq, d = q.shape
+    Hkv = np.asarray(k_pool).shape[2]
+    o = np.zeros((total_q, Hq, np.asarray(v_pool).shape[-1]), dtype=np.float64)
+    lse = np.zeros((total_q, Hq), dtype=np.float64)
+    for s in range(len(seq_lens)):
+        q0, q_len, ctx = _chunk_bounds(cu_seqlens_q, seq_lens, s)
+        if q_len == 0:
+            continue
+        L = int(seq_lens[s])
+        ks = _f64(gather_paged_kv(k_pool, block_table[s], L, page_size))
+        vs = _f64(gather_paged_kv(v_pool, block_table[s], L, page_size))
+        for h in range(Hq):
+            hk = gqa_kv_head(h, Hq, Hkv)
+            o_h, l_h = attention_head(q[q0:q0 + q_len, h], ks[:, hk], vs[:, hk], scale, causal, row_offset=ctx)
+            o[q0:q0 + q_len, h] = o_h
+            lse[q0:q0 + q_len, h] = l_h
     return o, lse

@@ -305,6 +305,120 @@ def pin_window_sdpa(o):
             assert abs(out[0, 0, r, t] - want) < 1e-12
 
 
+# -- appending to the paged cache and chunked prefill ----------------------------
+
+def pin_append_example(o):
+    """The pages' block table with 16-token blocks: a sequence holding 20
+    tokens receives 30 more.  Each new row must land at the (page, slot)
+    worked out by hand in the golden file; nothing else may change."""
+    with open(os.path.join(GOLDEN, "append_example.json")) as f:
+        ex = json.load(f)
+    ps, phys = ex["page_size"], ex["physical_blocks"]
+    ctx, n_new = ex["context_tokens"], ex["new_tokens"]
+    num_pages = 32
+    # label old slots (page, slot, 0) and new rows (-1, i, 1)
+    kp = np.zeros((num_pages, ps, 1, 3), dtype=np.int64)
+    for pg in range(num_pages):
+        for sl in range(ps):
+            kp[pg, sl, 0] = (pg, sl, 0)
+    vp = kp.copy()
+    kn = np.array([[[-1, i, 1]] for i in range(n_new)], dtype=np.int64)
+    vn = kn.copy()
+    table = np.array([phys], dtype=np.int32)
+    ko, vo = o.paged_append(kp, vp, kn, vn, table, np.array([0, n_new]), np.array([ctx + n_new]), ps)
+    for d in ex["destinations"]:
+        assert tuple(ko[d["physical_page"], d["slot"], 0]) == (-1, d["new_token"], 1)
+        assert tuple(vo[d["physical_page"], d["slot"], 0]) == (-1, d["new_token"], 1)
+    changed = {(pg, sl) for pg in range(num_pages) for sl in range(ps) if ko[pg, sl, 0, 2] == 1}
+    assert len(changed) == n_new
+    for sl in range(16):
+        assert tuple(ko[17, sl, 0]) == (17, sl, 0)
+    for sl in range(4):
+        assert tuple(ko[4, sl, 0]) == (4, sl, 0)
+    for sl in range(2, 16):
+        assert tuple(ko[8, sl, 0]) == (8, sl, 0)
+    assert np.array_equal(kp[:, :, :, 2], np.zeros_like(kp[:, :, :, 2]))  # inputs untouched
+
+
+def _chunked_setup(seed, lens, q_lens, ps, Hq, Hkv, d, num_pages):
+    rng = _rng(seed)
+    pool_k = _rand(rng, num_pages, ps, Hkv, d)
+    pool_v = _rand(rng, num_pages, ps, Hkv, d)
+    order = rng.permutation(num_pages)
+    width = max(-(-L // ps) for L in lens)
+    table = -np.ones((len(lens), width), dtype=np.int32)
+    used = 0
+    for s, L in enumerate(lens):
+        n = -(-L // ps)
+        table[s, :n] = order[used:used + n]
+        used += n
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int64)
+    q = _rand(rng, int(cu[-1]), Hq, d)
+    return q, pool_k, pool_v, table, cu
+
+
+def pin_paged_prefill_sdpa(o):
+    """Chunked prefill against PyTorch's fp64 SDPA with an explicit mask in
+    which new query i of a sequence with ctx cached tokens sees keys
+    0..ctx+i (and, without the causal mask, all keys)."""
+    lens, q_lens = [9, 23, 5, 17, 1], [9, 6, 1, 17, 1]
+    ps, Hq, Hkv, d = 4, 4, 2, 8
+    q, pk, pv, table, cu = _chunked_setup(30, lens, q_lens, ps, Hq, Hkv, d, 24)
+    for causal in (True, False):
+        out, lse = o.paged_prefill(q, pk, pv, table, cu, np.array(lens), ps, 0.3, causal)
+        for s, L in enumerate(lens):
+            ql, ctx = q_lens[s], L - q_lens[s]
+            kc = np.stack([pk[table[s, t // ps], t % ps] for t in range(L)])
+            vc = np.stack([pv[table[s, t // ps], t % ps] for t in range(L)])
+            tq = torch.from_numpy(q[cu[s]:cu[s + 1]].transpose(1, 0, 2))            # [Hq, ql, d]
+            tk = torch.from_numpy(kc.transpose(1, 0, 2)).repeat_interleave(Hq // Hkv, 0)
+            tv = torch.from_numpy(vc.transpose(1, 0, 2)).repeat_interleave(Hq // Hkv, 0)
+            i = torch.arange(ql)[:, None]
+            j = torch.arange(L)[None, :]
+            allowed = (j <= ctx + i) if causal else torch.ones(ql, L, dtype=torch.bool)
+            ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=allowed, scale=0.3)
+            ref_lse = torch.logsumexp((0.3 * (tq @ tk.transpose(-1, -2))).masked_fill(~allowed, float("-inf")), -1)
+            assert np.max(np.abs(out[cu[s]:cu[s + 1]] - ref.numpy().transpose(1, 0, 2))) < 1e-12
+            assert np.max(np.abs(lse[cu[s]:cu[s + 1]] - ref_lse.numpy().T)) < 1e-12
+
+
+def pin_paged_prefill_brute(o):
+    """Scalar brute force, ratio form: the new query i of a sequence with
+    ctx = 3 cached tokens averages V over keys 0..3+i with weights
+    exp(scale q.k)."""
+    lens, q_lens = [7], [4]
+    ps, Hq, Hkv, d = 2, 2, 1, 4
+    q, pk, pv, table, cu = _chunked_setup(31, lens, q_lens, ps, Hq, Hkv, d, 6)
+    out, lse = o.paged_prefill(q, pk, pv, table, cu, np.array(lens), ps, 0.5, True)
+    for i in range(4):
+        for h in range(Hq):
+            keys = range(0, 3 + i + 1)
+            w = [math.exp(0.5 * math.fsum(float(q[i, h, c]) * float(pk[table[0, t // ps], t % ps, 0, c])
+                                          for c in range(d))) for t in keys]
+            z = math.fsum(w)
+            for c in range(d):
+                want = math.fsum(wt * float(pv[table[0, t // ps], t % ps, 0, c]) for wt, t in zip(w, keys)) / z
+                assert abs(out[i, h, c] - want) < 1e-12
+            assert abs(lse[i, h] - math.log(z)) < 1e-12
+
+
+def pin_chunked_equals_whole(o):
+    """A sequence prefilled in one chunk, or as a first chunk followed by a
+    second one over the cache the first left behind, gives the same rows: a
+    row depends only on its own position and keys."""
+    L, a, ps, Hq, Hkv, d = 21, 8, 4, 2, 2, 8
+    q, pk, pv, table, _ = _chunked_setup(32, [L], [L], ps, Hq, Hkv, d, 8)
+    whole_o, whole_l = o.paged_prefill(q, pk, pv, table, np.array([0, L]), np.array([L]), ps, 0.4, True)
+    first_o, first_l = o.paged_prefill(q[:a], pk, pv, table, np.array([0, a]), np.array([a]), ps, 0.4, True)
+    second_o, second_l = o.paged_prefill(q[a:], pk, pv, table, np.array([0, L - a]), np.array([L]), ps, 0.4,
+                                         True)
+    assert np.max(np.abs(whole_o[:a] - first_o)) < 1e-12 and np.max(np.abs(whole_l[:a] - first_l)) < 1e-12
+    assert np.max(np.abs(whole_o[a:] - second_o)) < 1e-12 and np.max(np.abs(whole_l[a:] - second_l)) < 1e-12
+    # the last row is the decode of the same sequence
+    dec_o, dec_l = o.paged_decode(q[L - 1:L], pk, pv, table, np.array([L]), ps, 0.4)
+    assert np.max(np.abs(whole_o[L - 1] - dec_o[0])) < 1e-12 and np.max(np.abs(whole_l[L - 1] - dec_l[0])) < 1e-12
+
+
 ALL_PINS = [
     pin_rows_sum_to_one,
     pin_constant_v,
@@ -318,4 +432,8 @@ ALL_PINS = [
     pin_printed_sizes,
     pin_window_closed_form,
     pin_window_sdpa,
+    pin_append_example,
+    pin_paged_prefill_sdpa,
+    pin_paged_prefill_brute,
+    pin_chunked_equals_whole,
 ]

@@ -194,6 +194,45 @@ def _mut_window_ignored(m):
         q, k, scale, causal, row_offset, None)
 
 
+def _mut_append_shifted(m):
+    orig = m.paged_append
+    def f(kp, vp, kn, vn, table, cu, lens, ps):
+        return orig(kp, vp, kn, vn, table, cu, np.asarray(lens) + 1, ps)  # writes one slot late
+    m.paged_append = f
+
+
+def _mut_append_ignores_table(m):
+    def f(kp, vp, kn, vn, table, cu, lens, ps):
+        kp, vp = np.array(kp, copy=True), np.array(vp, copy=True)
+        for s in range(len(lens)):
+            q0, ql = int(cu[s]), int(cu[s + 1]) - int(cu[s])
+            ctx = int(lens[s]) - ql
+            for i in range(ql):
+                t = ctx + i
+                kp[t // ps, t % ps] = np.asarray(kn)[q0 + i]
+                vp[t // ps, t % ps] = np.asarray(vn)[q0 + i]
+        return kp, vp
+    m.paged_append = f
+
+
+def _mut_prefill_no_offset(m):
+    orig = m.attention_head
+    def head(q, k, v, scale, causal, row_offset=0, window_left=None):
+        return orig(q, k, v, scale, causal, 0, window_left)
+    m.attention_head = head
+
+
+def _mut_prefill_queries_from_start(m):
+    """Takes the new queries as tokens 0..q_len-1 (top-left alignment)."""
+    orig = m.paged_prefill
+    def f(q, kp, vp, table, cu, lens, ps, scale, causal=True):
+        cu = np.asarray(cu)
+        ql = np.diff(cu)
+        o_, l_ = orig(q, kp, vp, table, cu, ql, ps, scale, causal)
+        return o_, l_
+    m.paged_prefill = f
+
+
 MUTANTS = [
     _mut_drop_scale,
     _mut_scale_squared,
@@ -209,6 +248,10 @@ MUTANTS = [
     _mut_page_no_table,
     _mut_window_off_by_one,
     _mut_window_ignored,
+    _mut_append_shifted,
+    _mut_append_ignores_table,
+    _mut_prefill_no_offset,
+    _mut_prefill_queries_from_start,
 ]
 
 
