@@ -53,6 +53,12 @@ SIGNATURES = {
     "paged_attn_decode_graph_launch": (_c_i, [_c_p, _c_p]),
     "paged_attn_decode_graph_destroy": (_c_i, [_c_p]),
     "attn_device_status": (_c_i, [_c_p, ctypes.POINTER(ctypes.c_uint)]),
+    "paged_kv_append": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
+                               _c_i, _c_p]),
+    "paged_prefill": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
+                             _c_i, _c_i, _c_i, _c_f, _c_p]),
+    "paged_prefill_append": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i,
+                                    _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p]),
 }
 
 # Size of the scratch array built into the library for paged_attn_decode_noalloc.
@@ -299,3 +305,97 @@ def device_status(stream=None) -> int:
     if rc not in (ATTN_OK, 7):
         raise AttnError(rc, "attn_device_status")
     return int(bits.value)
+
+
+def _paged_chunk_args(k_pool, v_pool, block_table, cu_seqlens_q, seq_lens):
+    _require(k_pool, "k_pool", torch.bfloat16, 4)
+    _require(v_pool, "v_pool", torch.bfloat16, 4)
+    _require(block_table, "block_table", torch.int32, 2)
+    _require(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _require(seq_lens, "seq_lens", torch.int32, 1)
+    if v_pool.shape != k_pool.shape:
+        raise ValueError("k_pool and v_pool differ in shape")
+    S = seq_lens.shape[0]
+    if cu_seqlens_q.shape[0] != S + 1 or block_table.shape[0] != S:
+        raise ValueError("cu_seqlens_q / block_table do not match the number of sequences")
+    num_pages, page_size, Hkv, d = k_pool.shape
+    return S, num_pages, page_size, Hkv, d, block_table.shape[1]
+
+
+def paged_kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                    block_table: torch.Tensor, cu_seqlens_q: torch.Tensor, seq_lens: torch.Tensor, stream=None):
+    """Write each sequence's new K/V rows (packed [total_q, Hkv, d] bf16,
+    rows cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1) into the paged pools at
+    logical tokens seq_lens[s] - q_len .. seq_lens[s] - 1.  In place."""
+    S, num_pages, page_size, Hkv, d, max_pages = _paged_chunk_args(k_pool, v_pool, block_table, cu_seqlens_q,
+                                                                   seq_lens)
+    _require(k_new, "k_new", torch.bfloat16, 3)
+    _require(v_new, "v_new", torch.bfloat16, 3)
+    total_q = k_new.shape[0]
+    if k_new.shape != (total_q, Hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("k_new / v_new do not match the pools")
+    rc = lib().paged_kv_append(k_new.data_ptr(), v_new.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+                               cu_seqlens_q.data_ptr(), seq_lens.data_ptr(), block_table.data_ptr(), S, total_q,
+                               Hkv, d, page_size, max_pages, num_pages, _stream_handle(stream))
+    _check(rc, "paged_kv_append")
+
+
+def _prefill_outputs(q, out, lse):
+    total_q, Hq, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((total_q, Hq), dtype=torch.float32, device=q.device)
+    _require(out, "out", torch.bfloat16, 3)
+    _require(lse, "lse", torch.float32, 2)
+    return out, lse
+
+
+def paged_prefill(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, block_table: torch.Tensor,
+                  cu_seqlens_q: torch.Tensor, seq_lens: torch.Tensor, causal: bool = True,
+                  scale: float | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                  stream=None):
+    """Chunked prefill over a paged cache: q [total_q, Hq, d] bf16 packed by
+    sequence; new query i of sequence s is token seq_lens[s] - q_len + i.
+    Returns (o [total_q, Hq, d] bf16, lse [total_q, Hq] fp32)."""
+    S, num_pages, page_size, Hkv, d, max_pages = _paged_chunk_args(k_pool, v_pool, block_table, cu_seqlens_q,
+                                                                   seq_lens)
+    _require(q, "q", torch.bfloat16, 3)
+    total_q, Hq, dq = q.shape
+    if dq != d:
+        raise ValueError("q and the pools differ in head dim")
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    out, lse = _prefill_outputs(q, out, lse)
+    rc = lib().paged_prefill(q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), cu_seqlens_q.data_ptr(),
+                             seq_lens.data_ptr(), block_table.data_ptr(), out.data_ptr(), lse.data_ptr(), S, total_q,
+                             Hq, Hkv, d, page_size, max_pages, num_pages, int(bool(causal)), float(scale),
+                             _stream_handle(stream))
+    _check(rc, "paged_prefill")
+    return out, lse
+
+
+def paged_prefill_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_pool: torch.Tensor,
+                         v_pool: torch.Tensor, block_table: torch.Tensor, cu_seqlens_q: torch.Tensor,
+                         seq_lens: torch.Tensor, causal: bool = True, scale: float | None = None,
+                         out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """paged_kv_append then paged_prefill in one call (the pools are
+    updated in place).  Returns (o, lse) as paged_prefill does."""
+    S, num_pages, page_size, Hkv, d, max_pages = _paged_chunk_args(k_pool, v_pool, block_table, cu_seqlens_q,
+                                                                   seq_lens)
+    _require(q, "q", torch.bfloat16, 3)
+    _require(k_new, "k_new", torch.bfloat16, 3)
+    _require(v_new, "v_new", torch.bfloat16, 3)
+    total_q, Hq, dq = q.shape
+    if dq != d or k_new.shape != (total_q, Hkv, d) or v_new.shape != k_new.shape:
+        raise ValueError("q / k_new / v_new do not match the pools")
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    out, lse = _prefill_outputs(q, out, lse)
+    rc = lib().paged_prefill_append(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_pool.data_ptr(),
+                                    v_pool.data_ptr(), cu_seqlens_q.data_ptr(), seq_lens.data_ptr(),
+                                    block_table.data_ptr(), out.data_ptr(), lse.data_ptr(), S, total_q, Hq, Hkv, d,
+                                    page_size, max_pages, num_pages, int(bool(causal)), float(scale),
+                                    _stream_handle(stream))
+    _check(rc, "paged_prefill_append")
+    return out, lse

@@ -14,6 +14,7 @@
 
 #include "attn_b200.h"
 #include "decode_sm100.cuh"
+#include "paged_append.cuh"
 #include "prefill_sm100.cuh"
 
 namespace {
@@ -92,17 +93,18 @@ int sm_count() {
   return counts[dev];
 }
 
-template <int D, bool CAUSAL, bool WINDOW>
+template <int D, bool CAUSAL, bool WINDOW, bool PAGED = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const attn::PrefillParams& p, cudaStream_t stream) {
-  using L = attn::PrefillLayout<D>;
-  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, WINDOW>;
-  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL, WINDOW>>(L::kAlloc);
+  using L = attn::PrefillLayout<D, PAGED>;
+  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED>;
+  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED>>(L::kAlloc);
   if (e != cudaSuccess) return fail_cuda(e);
   const int sms = sm_count();
   if (sms <= 0) return fail_cuda(cudaErrorInvalidDevice);
-  // Persistent: one CTA per SM (or per work item when there are fewer).
-  const unsigned grid = static_cast<unsigned>(p.num_items < sms ? p.num_items : sms);
+  // Persistent: one CTA per SM (or per work item when there are fewer; the
+  // paged kernels count their items on the device and always take one per SM).
+  const unsigned grid = static_cast<unsigned>(PAGED || p.num_items >= sms ? sms : p.num_items);
   kernel<<<grid, attn::kPrefillThreads, L::kAlloc, stream>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail_cuda(e);
@@ -463,6 +465,180 @@ int attn_device_status(void* stream, unsigned int* bits) {
     return ATTN_ERR_DEVICE;
   }
   return ATTN_OK;
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Appending to a paged cache, and chunked prefill over it
+// ----------------------------------------------------------------------------
+
+namespace {
+
+constexpr int kAppendBlocksPerSm = 16;
+
+bool page_size_supported(int page_size) {
+  return page_size == 16 || page_size == 32 || page_size == 64 || page_size == 128 || page_size == 256;
+}
+
+bool misaligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) != 0; }
+
+// Checks shared by the append and the chunked prefill (no CUDA call).
+int validate_paged_cache(const void* k_pool, const void* v_pool, const int32_t* cu_seqlens_q,
+                         const int32_t* seq_lens, const int32_t* block_table, int num_seqs, int total_q, int Hkv,
+                         int d, int page_size, int max_pages, int num_pages) {
+  if (!k_pool || !v_pool || !cu_seqlens_q || !seq_lens || !block_table) return ATTN_ERR_NULL;
+  if (num_seqs < 1 || total_q < 0 || Hkv < 1 || max_pages < 1 || num_pages < 1 || page_size < 1)
+    return ATTN_ERR_SHAPE;
+  if (d != 64 && d != 128) return ATTN_ERR_SHAPE;
+  if (Hkv > 65535) return ATTN_ERR_SHAPE;
+  if (static_cast<long long>(num_pages) * page_size > INT_MAX ||
+      static_cast<long long>(max_pages) * page_size > INT_MAX ||
+      static_cast<long long>(num_seqs) * max_pages > INT_MAX)
+    return ATTN_ERR_SHAPE;
+  if (!page_size_supported(page_size)) return ATTN_ERR_UNSUPPORTED;
+  if (misaligned16(k_pool) || misaligned16(v_pool) || misaligned4(cu_seqlens_q) || misaligned4(seq_lens) ||
+      misaligned4(block_table))
+    return ATTN_ERR_ALIGN;
+  return ATTN_OK;
+}
+
+int validate_paged_prefill(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                           const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table,
+                           attn_bf16* o, float* lse, int num_seqs, int total_q, int Hq, int Hkv, int d,
+                           int page_size, int max_pages, int num_pages, int causal, float scale) {
+  if (!q || !o || !lse) return ATTN_ERR_NULL;
+  const int st = validate_paged_cache(k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, num_seqs, total_q, Hkv,
+                                      d, page_size, max_pages, num_pages);
+  if (st != ATTN_OK) return st;
+  if (Hq < 1 || Hq % Hkv != 0 || Hq > 65535) return ATTN_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return ATTN_ERR_SHAPE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_SHAPE;
+  if (static_cast<long long>(total_q) * Hq > INT_MAX) return ATTN_ERR_SHAPE;
+  if (num_seqs > attn::kPagedMaxSeqs) return ATTN_ERR_UNSUPPORTED;
+  if (misaligned16(q) || misaligned16(o) || misaligned4(lse)) return ATTN_ERR_ALIGN;
+  return ATTN_OK;
+}
+
+int launch_append(const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_pool, attn_bf16* v_pool,
+                  const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table, int num_seqs,
+                  int total_q, int Hkv, int d, int page_size, int max_pages, int num_pages, cudaStream_t stream) {
+  if (total_q == 0) return ATTN_OK;
+  const int sms = sm_count();
+  if (sms <= 0) return fail_cuda(cudaErrorInvalidDevice);
+  attn::AppendParams p;
+  p.k_new = reinterpret_cast<const __nv_bfloat16*>(k_new);
+  p.v_new = reinterpret_cast<const __nv_bfloat16*>(v_new);
+  p.k_pool = reinterpret_cast<__nv_bfloat16*>(k_pool);
+  p.v_pool = reinterpret_cast<__nv_bfloat16*>(v_pool);
+  p.cu_q = cu_seqlens_q;
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.num_seqs = num_seqs;
+  p.total_q = total_q;
+  p.Hkv = Hkv;
+  p.D = d;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+  constexpr int kWarps = attn::kAppendThreads / 32;  // one new token per warp
+  const long long want = (static_cast<long long>(total_q) + kWarps - 1) / kWarps;
+  const long long cap = static_cast<long long>(sms) * kAppendBlocksPerSm;
+  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+  attn::paged_append_kernel<<<grid, attn::kAppendThreads, 0, stream>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ATTN_OK : fail_cuda(e);
+}
+
+int launch_paged_prefill(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                         const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table,
+                         attn_bf16* o, float* lse, int num_seqs, int total_q, int Hq, int Hkv, int d, int page_size,
+                         int max_pages, int num_pages, int causal, float scale, cudaStream_t stream) {
+  if (total_q == 0) return ATTN_OK;
+  const int box_rows = page_size < 128 ? page_size : 128;
+  CUtensorMap tq, tk, tv;
+  const uint64_t d2 = static_cast<uint64_t>(d) * 2;
+  // Q: (d, packed token, head); pools: (d, page * page_size + slot, kv head).
+  if (!encode_3d(&tq, q, d, static_cast<uint64_t>(total_q), Hq, static_cast<uint64_t>(Hq) * d2, d2, 64, 128, 1) ||
+      !encode_3d(&tk, k_pool, d, static_cast<uint64_t>(num_pages) * page_size, Hkv, static_cast<uint64_t>(Hkv) * d2,
+                 d2, 64, static_cast<uint32_t>(box_rows), 1) ||
+      !encode_3d(&tv, v_pool, d, static_cast<uint64_t>(num_pages) * page_size, Hkv, static_cast<uint64_t>(Hkv) * d2,
+                 d2, 64, static_cast<uint32_t>(box_rows), 1))
+    return fail_cuda(cudaErrorInvalidValue);
+  attn::PrefillParams p{};
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = 1;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = 0;
+  p.group = Hq / Hkv;
+  p.num_m = 0;
+  p.num_items = 0;
+  p.window_left = -1;
+  p.scale_log2 = scale * kLog2e;
+  p.cu_q = cu_seqlens_q;
+  p.seq_lens = seq_lens;
+  p.block_table = block_table;
+  p.k_pool = reinterpret_cast<const __nv_bfloat16*>(k_pool);
+  p.v_pool = reinterpret_cast<const __nv_bfloat16*>(v_pool);
+  p.num_seqs = num_seqs;
+  p.total_q = total_q;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.page_size = page_size;
+  p.page_box = box_rows;
+  if (d == 128)
+    return causal ? launch_prefill<128, true, false, true>(tq, tk, tv, p, stream)
+                  : launch_prefill<128, false, false, true>(tq, tk, tv, p, stream);
+  return causal ? launch_prefill<64, true, false, true>(tq, tk, tv, p, stream)
+                : launch_prefill<64, false, false, true>(tq, tk, tv, p, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_kv_append(const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_pool, attn_bf16* v_pool,
+                    const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table, int num_seqs,
+                    int total_q, int Hkv, int d, int page_size, int max_pages, int num_pages, void* stream) {
+  const int st = validate_paged_cache(k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, num_seqs, total_q, Hkv,
+                                      d, page_size, max_pages, num_pages);
+  if (st != ATTN_OK) return st;
+  if (total_q > 0 && (!k_new || !v_new)) return ATTN_ERR_NULL;
+  if (total_q > 0 && (misaligned16(k_new) || misaligned16(v_new))) return ATTN_ERR_ALIGN;
+  return launch_append(k_new, v_new, k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, num_seqs, total_q, Hkv, d,
+                       page_size, max_pages, num_pages, static_cast<cudaStream_t>(stream));
+}
+
+int paged_prefill(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                  const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table, attn_bf16* o,
+                  float* lse, int num_seqs, int total_q, int Hq, int Hkv, int d, int page_size, int max_pages,
+                  int num_pages, int causal, float scale, void* stream) {
+  const int st = validate_paged_prefill(q, k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, o, lse, num_seqs,
+                                        total_q, Hq, Hkv, d, page_size, max_pages, num_pages, causal, scale);
+  if (st != ATTN_OK) return st;
+  return launch_paged_prefill(q, k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, o, lse, num_seqs, total_q, Hq,
+                              Hkv, d, page_size, max_pages, num_pages, causal, scale,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int paged_prefill_append(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_pool,
+                         attn_bf16* v_pool, const int32_t* cu_seqlens_q, const int32_t* seq_lens,
+                         const int32_t* block_table, attn_bf16* o, float* lse, int num_seqs, int total_q, int Hq,
+                         int Hkv, int d, int page_size, int max_pages, int num_pages, int causal, float scale,
+                         void* stream) {
+  const int st = validate_paged_prefill(q, k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, o, lse, num_seqs,
+                                        total_q, Hq, Hkv, d, page_size, max_pages, num_pages, causal, scale);
+  if (st != ATTN_OK) return st;
+  if (total_q > 0 && (!k_new || !v_new)) return ATTN_ERR_NULL;
+  if (total_q > 0 && (misaligned16(k_new) || misaligned16(v_new))) return ATTN_ERR_ALIGN;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int a = launch_append(k_new, v_new, k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, num_seqs, total_q,
+                              Hkv, d, page_size, max_pages, num_pages, s);
+  if (a != ATTN_OK) return a;
+  return launch_paged_prefill(q, k_pool, v_pool, cu_seqlens_q, seq_lens, block_table, o, lse, num_seqs, total_q, Hq,
+                              Hkv, d, page_size, max_pages, num_pages, causal, scale, s);
 }
 
 }  // extern "C"

@@ -60,21 +60,33 @@ __device__ __forceinline__ float exp2_poly(float x) {
 }
 
 struct PrefillParams {
-  __nv_bfloat16* o;  // [B, Hq, N, D]
-  float* lse;        // [B, Hq, N]
+  __nv_bfloat16* o;  // [B, Hq, N, D]; paged: [total_q, Hq, D]
+  float* lse;        // [B, Hq, N];    paged: [total_q, Hq]
   int B, Hq, Hkv, N;
   int group;         // Hq / Hkv
   int num_m;         // ceil(N / 256): 256-row query blocks per head
-  int num_items;     // B * Hq * num_m
+  int num_items;     // B * Hq * num_m (paged: counted on the device)
   int window_left;   // query i sees keys >= i - window_left (kernels with WINDOW only)
   float scale_log2;  // scale * log2(e)
+  // Paged prefill (kernels with PAGED only): the new queries of sequence s
+  // are packed rows cu_q[s] .. cu_q[s+1]-1; the cache holds seq_lens[s]
+  // tokens of it (the new ones last), read through block_table.
+  const int32_t* cu_q;         // [num_seqs + 1]
+  const int32_t* seq_lens;     // [num_seqs]
+  const int32_t* block_table;  // [num_seqs, max_pages]
+  const __nv_bfloat16* k_pool; // [num_pages, page_size, Hkv, D] (plain loads of partial pages)
+  const __nv_bfloat16* v_pool;
+  int num_seqs, total_q, max_pages, num_pages, page_size;
+  int page_box;                // rows per K/V TMA box: min(page_size, 128)
 };
+
+constexpr int kPagedMaxSeqs = 1024;  // sequences per paged-prefill call
 
 constexpr int kPrefillThreads = 512;
 constexpr float kRescaleThreshold = 8.0f;  // in log2 units
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D>
+template <int D, bool PAGED = false>
 struct PrefillLayout {
   static constexpr int NS = 2;                 // K and V ring depth
   static constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128B-swizzled box)
@@ -85,7 +97,11 @@ struct PrefillLayout {
   static constexpr int kV = kK + NS * kTileBytes;
   static constexpr int kStats = kV + NS * kTileBytes;  // float [tile 2][slot 2][m,l][128 rows]
   static constexpr int kStatsBytes = 2 * 2 * 2 * 128 * 4;
-  static constexpr int kBar = kStats + kStatsBytes;
+  // Paged: per-sequence table cached at kernel start: item offsets [S+1],
+  // cu_q [S+1], seq_lens [S], and 16 ints of scan scratch.
+  static constexpr int kSeq = kStats + kStatsBytes;
+  static constexpr int kSeqBytes = PAGED ? (3 * kPagedMaxSeqs + 2 + 16) * 4 : 0;
+  static constexpr int kBar = (kSeq + kSeqBytes + 7) / 8 * 8;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarQEmpty = 1;
   static constexpr int kBarKFull = 2;
@@ -110,21 +126,71 @@ struct PrefillLayout {
 // One work item: 256 query rows [m*256, m*256+256) of head (b, h).  Query
 // tile t (rows m*256 + 128t ...) sees the 128-key KV tiles j with
 // lo[t] <= j < hi[t]; the item walks j over [jb, je), the union of both.
+// Paged: b is the sequence, its new queries are packed rows q0 .. q0+n_q-1,
+// query row r is token pos0 + r of a cache of n_kv tokens.
 struct PrefillItem {
   int b, h, m;
   int lo0, hi0, lo1, hi1;  // tile 1 is empty (lo1 = hi1) when its rows lie past N
   int jb, je;
+  int q0, n_q, n_kv, pos0;  // paged only
   __device__ __forceinline__ int lo(int t) const { return t ? lo1 : lo0; }
   __device__ __forceinline__ int hi(int t) const { return t ? hi1 : hi0; }
   __device__ __forceinline__ bool active(int t, int j) const { return lo(t) <= j && j < hi(t); }
   __device__ __forceinline__ bool has(int t) const { return hi(t) > lo(t); }
 };
 
-template <bool CAUSAL, bool WINDOW>
-__device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, PrefillItem& it) {
+// Sequence table of the paged kernels, in shared memory.
+struct PagedSeqs {
+  const int* item_off;  // [S + 1]: first item of each sequence, item_off[S] = total
+  const int* cu_q;      // [S + 1]
+  const int* lens;      // [S]
+};
+
+template <bool CAUSAL>
+__device__ __forceinline__ bool paged_item(int idx, const PrefillParams& p, const PagedSeqs& sq,
+                                           PrefillItem& it) {
+  if (idx >= sq.item_off[p.num_seqs]) return false;
+  int lo = 0, hi = p.num_seqs;  // item_off[lo] <= idx < item_off[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (sq.item_off[mid] <= idx) lo = mid; else hi = mid;
+  }
+  const int local = idx - sq.item_off[lo];
+  it.b = lo;
+  it.q0 = sq.cu_q[lo];
+  it.n_q = sq.cu_q[lo + 1] - it.q0;
+  it.n_kv = sq.lens[lo];
+  it.pos0 = it.n_kv - it.n_q;
+  const int n_m = (it.n_q + 255) / 256;
+  it.h = local % p.Hq;
+  const int rank = local / p.Hq;  // 0 = heaviest (causal)
+  it.m = CAUSAL ? (n_m - 1 - rank) : rank;
+  {
+    const int r0 = it.pos0 + it.m * 256;
+    const int last_key = CAUSAL ? min(r0 + 127, it.n_kv - 1) : it.n_kv - 1;
+    it.lo0 = 0;
+    it.hi0 = last_key / 128 + 1;
+  }
+  if (it.m * 256 + 128 >= it.n_q) {
+    it.lo1 = it.hi1 = 0;
+  } else {
+    const int r0 = it.pos0 + it.m * 256 + 128;
+    const int last_key = CAUSAL ? min(r0 + 127, it.n_kv - 1) : it.n_kv - 1;
+    it.lo1 = 0;
+    it.hi1 = last_key / 128 + 1;
+  }
+  it.jb = 0;
+  it.je = max(it.hi0, it.hi1);
+  return true;
+}
+
+template <bool CAUSAL, bool WINDOW, bool PAGED = false>
+__device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, PrefillItem& it,
+                                             const PagedSeqs& sq = PagedSeqs{}) {
   const int G = static_cast<int>(gridDim.x);
   const int c = static_cast<int>(blockIdx.x);
   const int idx = round * G + ((round & 1) ? (G - 1 - c) : c);
+  if constexpr (PAGED) return paged_item<CAUSAL>(idx, p, sq, it);
   if (idx >= p.num_items) return false;
   const int bh_count = p.B * p.Hq;
   const int rank = idx / bh_count;  // 0 = heaviest
@@ -157,6 +223,60 @@ __device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, 
   return true;
 }
 
+// Paged kernels: every CTA caches the sequence table in shared memory and
+// counts the work items of each sequence (ceil(q_len / 256) query blocks per
+// head) with a block-wide prefix sum.  A sequence whose lengths are out of
+// range gets no items and sets kErrPagedTable.  Called by all threads.
+__device__ __forceinline__ void paged_seq_table(const PrefillParams& p, int* off, int* cuq, int* lens,
+                                                int* scratch) {
+  const int S = p.num_seqs;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nw = static_cast<int>(blockDim.x >> 5);
+  int v[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    const int s = 2 * static_cast<int>(threadIdx.x) + e;
+    v[e] = 0;
+    if (s < S) {
+      const int a = p.cu_q[s], b = p.cu_q[s + 1], len = p.seq_lens[s];
+      cuq[s] = a;
+      lens[s] = len;
+      if (s == S - 1) cuq[S] = b;
+      const int nq = b - a;
+      if (a < 0 || nq < 0 || b > p.total_q || nq > len || len > p.max_pages * p.page_size) {
+        if (blockIdx.x == 0) atomicOr(&g_attn_device_error, kErrPagedTable);
+      } else {
+        v[e] = (nq + 255) / 256 * p.Hq;
+      }
+    }
+  }
+  const int tot = v[0] + v[1];
+  int x = tot;  // inclusive scan over the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) scratch[lane] = w;
+  }
+  __syncthreads();
+  const int before = x - tot + (warp > 0 ? scratch[warp - 1] : 0);
+  const int s0 = 2 * static_cast<int>(threadIdx.x);
+  if (s0 < S) off[s0] = before;
+  if (s0 + 1 < S) off[s0 + 1] = before + v[0];
+  if (threadIdx.x == 0) off[S] = scratch[nw - 1];
+}
+
 // Register split per warpgroup (launch: 512 threads x 128 registers):
 // softmax 2 x 184, epilogue 64, producer/MMA 80 -> 4 x 128 per lane slot.
 __device__ __forceinline__ void reg_alloc_softmax() {
@@ -169,13 +289,14 @@ __device__ __forceinline__ void reg_alloc_control() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
 }
 
-template <int D, bool CAUSAL, bool WINDOW>
+template <int D, bool CAUSAL, bool WINDOW, bool PAGED>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
   static_assert(D == 64 || D == 128, "head dim");
-  using L = PrefillLayout<D>;
+  static_assert(!(PAGED && WINDOW), "the paged kernels have no window");
+  using L = PrefillLayout<D, PAGED>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -187,6 +308,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int wg = warp >> 2;
+
+  PagedSeqs sq{};
+  if constexpr (PAGED) {
+    int* off = reinterpret_cast<int*>(smem + L::kSeq);
+    int* cuq = off + kPagedMaxSeqs + 1;
+    int* lens = cuq + kPagedMaxSeqs + 1;
+    paged_seq_table(p, off, cuq, lens, lens + kPagedMaxSeqs);
+    sq = PagedSeqs{off, cuq, lens};
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarQFull), 1);
@@ -226,48 +356,121 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   if (wg == 3) {
     reg_alloc_control();
-    if (warp == 12 && lane == 0) {
+    if (warp == 12) {
       // ---------------------------------------------------------- producer
+      // Lane 0 waits and issues the copies; the paged kernels also use the
+      // other lanes for block-table lookups and the partly used last page.
       int kv_it = 0, k_issued = 0, v_issued = 0, q_issued = 0;
       bool ok = true;
-      PrefillItem it;
+      PrefillItem it{};
+      auto wait0 = [&](uint32_t b, uint32_t parity, unsigned int code) -> bool {
+        int r = 1;
+        if (lane == 0) r = mbar_wait(b, parity, code) ? 1 : 0;
+        return __shfl_sync(0xffffffffu, r, 0) != 0;
+      };
+      // Keys 128j .. 128j+127 of K or V into the stage at dst.
+      auto load_tile = [&](const CUtensorMap* map, const __nv_bfloat16* pool, uint32_t dst, uint32_t full, int j,
+                           int kz) {
+        if constexpr (!PAGED) {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(full, L::kTileBytes);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(dst + c * L::kBoxBytes, map, full, c * 64, j * 128, kz);
+          }
+        } else {
+          // Box b (lane b) holds keys 128j + b*pb ...: a page (or a 128-key
+          // part of one) found through the block table.  Boxes wholly past the
+          // sequence start outside the pool, so TMA fills them with zeros.
+          const int pb = p.page_box;
+          const int nbox = 128 / pb;
+          int row = p.num_pages * p.page_size;
+          int valid = pb;  // rows of the box inside the sequence
+          if (lane < nbox) {
+            const int pos = j * 128 + lane * pb;
+            if (pos < it.n_kv) {
+              int pg = p.block_table[static_cast<size_t>(it.b) * p.max_pages + pos / p.page_size];
+              if (pg < 0 || pg >= p.num_pages) {
+                atomicOr(&g_attn_device_error, kErrPagedTable);
+                pg = 0;  // keep every copy inside the pool; the result is flagged invalid
+              }
+              row = pg * p.page_size + pos % p.page_size;
+              valid = min(pb, it.n_kv - pos);
+            }
+          }
+          // The box with the sequence's last token, when only part of it is
+          // used, comes through plain loads: the slots past the end may hold
+          // anything (even NaN), so they are written as zeros instead.
+          const unsigned part = __ballot_sync(0xffffffffu, lane < nbox && valid < pb);
+          if (part != 0u) {
+            const int b = __ffs(part) - 1;
+            const int prow = __shfl_sync(0xffffffffu, row, b);
+            const int pval = __shfl_sync(0xffffffffu, valid, b);
+            constexpr int kChunks = (D / 64) * 8;  // 16-byte chunks per row
+            for (int idx = lane; idx < pb * kChunks; idx += 32) {
+              const int r = idx / kChunks;
+              const int c = (idx % kChunks) / 8;   // 64-column half
+              const int ch = idx % 8;              // chunk within the 128-byte row
+              const int tr = b * pb + r;           // row within the tile
+              uint4 val = make_uint4(0u, 0u, 0u, 0u);
+              if (r < pval)
+                val = *reinterpret_cast<const uint4*>(
+                    pool + ((static_cast<size_t>(prow + r) * p.Hkv + kz) * D + c * 64 + ch * 8));
+              const uint32_t a = dst + static_cast<uint32_t>(c * L::kBoxBytes + tr * 128 + ((ch ^ (tr & 7)) << 4));
+              *reinterpret_cast<uint4*>(smem + (a - base)) = val;
+            }
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+          const int ntma = nbox - (part != 0u ? 1 : 0);
+          if (lane == 0) {
+            if (ntma > 0)
+              mbar_arrive_expect_tx(full, static_cast<uint32_t>(ntma * pb * 128 * (D / 64)));
+            else
+              mbar_arrive(full);
+          }
+          for (int b = 0; b < nbox; ++b) {
+            const int rb = __shfl_sync(0xffffffffu, row, b);
+            if (lane == 0 && ((part >> b) & 1u) == 0u)
+              for (int c = 0; c < D / 64; ++c)
+                tma_load_3d(dst + static_cast<uint32_t>(c * L::kBoxBytes + b * pb * 128), map, full, c * 64, rb,
+                            kz);
+          }
+        }
+      };
       auto load_k = [&](int j, int kz) -> bool {
         const int st = kv_it % NS;
         const uint32_t round = static_cast<uint32_t>(kv_it / NS);
-        if (round > 0 && !mbar_wait(bar(L::kBarKEmpty + st), (round - 1) & 1u, kErrWaitKEmpty)) return false;
-        mbar_arrive_expect_tx(bar(L::kBarKFull + st), L::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(base + L::kK + st * L::kTileBytes + c * L::kBoxBytes, &tm_k, bar(L::kBarKFull + st),
-                      c * 64, j * 128, kz);
+        if (round > 0 && !wait0(bar(L::kBarKEmpty + st), (round - 1) & 1u, kErrWaitKEmpty)) return false;
+        load_tile(&tm_k, p.k_pool, base + L::kK + st * L::kTileBytes, bar(L::kBarKFull + st), j, kz);
         ++k_issued;
         return true;
       };
       auto load_v = [&](int j, int kz) -> bool {
         const int st = kv_it % NS;
         const uint32_t round = static_cast<uint32_t>(kv_it / NS);
-        if (round > 0 && !mbar_wait(bar(L::kBarVEmpty + st), (round - 1) & 1u, kErrWaitVEmpty)) return false;
-        mbar_arrive_expect_tx(bar(L::kBarVFull + st), L::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(base + L::kV + st * L::kTileBytes + c * L::kBoxBytes, &tm_v, bar(L::kBarVFull + st),
-                      c * 64, j * 128, kz);
+        if (round > 0 && !wait0(bar(L::kBarVEmpty + st), (round - 1) & 1u, kErrWaitVEmpty)) return false;
+        load_tile(&tm_v, p.v_pool, base + L::kV + st * L::kTileBytes, bar(L::kBarVFull + st), j, kz);
         ++v_issued;
         return true;
       };
-      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
-        const int qz = it.b * p.Hq + it.h;
-        const int kz = it.b * p.Hkv + it.h / p.group;  // GQA: consecutive query heads share a KV head
+      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
+        // Q rows: dense (d, row, b*Hq + h); paged (d, packed token, h).
+        const int qz = PAGED ? it.h : it.b * p.Hq + it.h;
+        const int qrow = (PAGED ? it.q0 : 0) + it.m * 256;
+        // GQA: consecutive query heads share a KV head
+        const int kz = (PAGED ? 0 : it.b * p.Hkv) + it.h / p.group;
         // The item's first K tile first: it can land while the previous item
         // still holds Q.
         if (!(ok = load_k(it.jb, kz))) break;
-        if (r > 0 && !(ok = mbar_wait(bar(L::kBarQEmpty), static_cast<uint32_t>(r - 1) & 1u, kErrWaitQ)))
-          break;
-        mbar_arrive_expect_tx(bar(L::kBarQFull), (it.has(1) ? 2 : 1) * L::kTileBytes);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(base + L::kQ0 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, it.m * 256, qz);
-        if (it.has(1))
+        if (r > 0 && !(ok = wait0(bar(L::kBarQEmpty), static_cast<uint32_t>(r - 1) & 1u, kErrWaitQ))) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar(L::kBarQFull), (it.has(1) ? 2 : 1) * L::kTileBytes);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(base + L::kQ1 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, it.m * 256 + 128,
-                        qz);
+            tma_load_3d(base + L::kQ0 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, qrow, qz);
+          if (it.has(1))
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(base + L::kQ1 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, qrow + 128, qz);
+        }
         ++q_issued;
         if (!(ok = load_v(it.jb, kz))) break;
         ++kv_it;
@@ -276,13 +479,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           if (!(ok = load_v(j, kz))) break;
         }
       }
-      // Every copy this thread started must land before the CTA may exit.
-      if (q_issued > 0)
-        mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(q_issued - 1) & 1u, kErrWaitDrain);
-      for (int j = max(0, k_issued - NS); j < k_issued; ++j)
-        mbar_wait(bar(L::kBarKFull + j % NS), static_cast<uint32_t>(j / NS) & 1u, kErrWaitDrain);
-      for (int j = max(0, v_issued - NS); j < v_issued; ++j)
-        mbar_wait(bar(L::kBarVFull + j % NS), static_cast<uint32_t>(j / NS) & 1u, kErrWaitDrain);
+      // Every copy this warp started must land before the CTA may exit.
+      if (lane == 0) {
+        if (q_issued > 0)
+          mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(q_issued - 1) & 1u, kErrWaitDrain);
+        for (int j = max(0, k_issued - NS); j < k_issued; ++j)
+          mbar_wait(bar(L::kBarKFull + j % NS), static_cast<uint32_t>(j / NS) & 1u, kErrWaitDrain);
+        for (int j = max(0, v_issued - NS); j < v_issued; ++j)
+          mbar_wait(bar(L::kBarVFull + j % NS), static_cast<uint32_t>(j / NS) & 1u, kErrWaitDrain);
+      }
+      __syncwarp();
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, false, false);
@@ -313,7 +519,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                       idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
       };
       PrefillItem it;
-      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
+      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
         if (!(ok = mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(r) & 1u, kErrWaitQ))) break;
         const int nkv = it.je - it.jb;
         {
@@ -392,7 +598,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t st_cnt[2] = {0u, 0u};  // items whose tile t this warpgroup has written out
     bool ok = true;
     PrefillItem it;
-    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
+    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (!it.has(t)) continue;
@@ -409,9 +615,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const float l_sum = sp[128 + row];
         mbar_arrive(bar(L::kBarStatsEmpty + 2 * t + slot));
         ++st_cnt[t];
-        const int grow = it.m * 256 + t * 128 + row;
+        const int grow = it.m * 256 + t * 128 + row;  // query row of the head (paged: of the sequence's chunk)
         const float inv_l = 1.f / l_sum;
-        const size_t row_index = static_cast<size_t>(it.b * p.Hq + it.h) * p.N + grow;
+        // O row / LSE index: dense [B, Hq, N, D] / [B, Hq, N]; paged by token, [total_q, Hq, D] / [total_q, Hq].
+        const bool valid = grow < (PAGED ? it.n_q : p.N);
+        const size_t row_index = PAGED ? (static_cast<size_t>(it.q0) + grow) * p.Hq + it.h
+                                       : static_cast<size_t>(it.b * p.Hq + it.h) * p.N + grow;
         __nv_bfloat16* orow = p.o + row_index * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -421,7 +630,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-          if (grow < p.N) {
+          if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -429,7 +638,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
           }
         }
-        if (grow < p.N) p.lse[row_index] = (m_used + log2f(l_sum)) * kLn2;
+        if (valid) p.lse[row_index] = (m_used + log2f(l_sum)) * kLn2;
         tc_fence_before();
         mbar_arrive(bar(L::kBarOFree + t));
       }
@@ -446,12 +655,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t s_cnt = 0, st_cnt = 0;
     bool ok = true;
     PrefillItem it;
-    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW>(r, p, it); ++r) {
+    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
       const int lo_t = it.lo(t);
       const int n_t = it.hi(t) - lo_t;  // KV tiles this query tile visits (>= 0)
       if (n_t == 0) continue;
-      const int row0 = it.m * 256 + t * 128;  // first row of this query tile
+      // Position (key index) of this tile's first query row; paged chunks
+      // start at the sequence's cached length.
+      const int row0 = (PAGED ? it.pos0 : 0) + it.m * 256 + t * 128;
       const int grow = row0 + row;
+      const int n_kv = PAGED ? it.n_kv : p.N;
       float m_used = -INFINITY;  // running max in scaled log2 units
       float l_sum = 0.f;
       for (int jj = 0; jj < n_t; ++jj) {
@@ -467,10 +679,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int kv0 = j * 128;
         // Tiles crossing the causal diagonal, a window's left edge or N get a
         // per-element mask (a select, so NaN-free -inf).
-        if ((CAUSAL && kv0 + 127 > row0) || kv0 + 128 > p.N ||
-            (WINDOW && kv0 < min(row0 + 127, p.N - 1) - p.window_left)) {
+        if ((CAUSAL && kv0 + 127 > row0) || kv0 + 128 > n_kv ||
+            (WINDOW && kv0 < min(row0 + 127, n_kv - 1) - p.window_left)) {
           // Visible keys of this row: [first, last], as offsets into the tile.
-          const int last = (CAUSAL ? min(grow, p.N - 1) : p.N - 1) - kv0;
+          const int last = (CAUSAL ? min(grow, n_kv - 1) : n_kv - 1) - kv0;
           if constexpr (WINDOW) {
             const int first = grow - p.window_left - kv0;
 #pragma unroll

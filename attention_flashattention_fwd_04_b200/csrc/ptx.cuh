@@ -32,6 +32,7 @@ enum : unsigned int {
   kErrWaitDrain = 1u << 9,
   kErrDecodeWait = 1u << 10,
   kErrDecodeTable = 1u << 11,
+  kErrPagedTable = 1u << 12,  // paged prefill / append: a length or block-table entry out of range
 };
 
 // Wall-clock limit for one wait (ns).  Real waits in these kernels last

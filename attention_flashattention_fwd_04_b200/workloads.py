@@ -16,6 +16,10 @@ rounded to nearest-even; draw order Q, K, V, then any per-position offset):
 * ``long_causal``  B=1, H=8, N=32768, d=128, causal, N(0,1) with one offset
   c_j ~ N(0, sigma=2) per key position added to every element of key row j
   (shared by all heads) to make peaked softmax rows, seed 5
+* ``chunked_prefill`` 16 sequences, Hq=32, Hkv=8, d=128, 16-token pages;
+  cached context lengths uniform in [0, 6144], new-chunk lengths uniform in
+  [256, 2048] (a serving step that appends a prompt chunk to each
+  sequence's cache and attends over all of it), seed 8
 * ``long_window``  the ``long_causal`` shapes and draws (seed 7) with a sliding
   window: query i sees keys i-4095 .. i (a 4096-key window, the size used by
   common sliding-window models; the pages name the pattern, not a size)
@@ -40,6 +44,11 @@ __all__ = [
     "DECODE_CONFIGS",
     "make_prefill_inputs",
     "make_decode_inputs",
+    "ChunkedConfig",
+    "CHUNKED_CONFIGS",
+    "make_chunked_inputs",
+    "chunked_flops",
+    "chunked_append_bytes",
     "prefill_flops",
     "visible_pairs",
     "decode_kv_bytes",
@@ -103,6 +112,116 @@ DECODE_CONFIGS = {
     # a small decode batch, where per-call host work and launch gaps dominate
     "small_decode": DecodeConfig("small_decode", 4, 32, 8, 128, 16, 256, 1024, 6),
 }
+
+
+@dataclass(frozen=True)
+class ChunkedConfig:
+    name: str
+    num_seqs: int
+    Hq: int
+    Hkv: int
+    d: int
+    page_size: int
+    ctx_range: tuple
+    q_range: tuple
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32))
+
+
+CHUNKED_CONFIGS = {
+    "chunked_prefill": ChunkedConfig("chunked_prefill", 16, 32, 8, 128, 16, (0, 6144), (256, 2048), 8),
+}
+
+
+def make_chunked_inputs(cfg: ChunkedConfig, device: str | torch.device = "cpu", poison: bool = False,
+                        ctx_lens=None, q_lens=None, spare_pages: int = 0):
+    """Inputs of one append + chunked-prefill step over a paged cache.
+
+    Sequence s holds ctx_s cached tokens and receives q_s new ones
+    (seq_len = ctx + q).  Returns a dict with q [total_q,Hq,d], k_new / v_new
+    [total_q,Hkv,d] (packed by sequence, cu_seqlens_q [S+1] int32), pools
+    [num_pages,page_size,Hkv,d] holding every sequence's context (pages for
+    all seq_len tokens are allocated up front, a seeded permutation of the
+    pool), block_table [S,width] int32 (-1 past each sequence's pages),
+    seq_lens [S] int32.  The slots of the new tokens and every slot past a
+    sequence's end hold NaN when ``poison`` (the append must overwrite the
+    former; nothing may read the latter), else random values.
+    ``spare_pages`` adds unused pages (filled like the rest) to the pool.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(cfg.seed)
+    S, ps = cfg.num_seqs, cfg.page_size
+    ctx = torch.randint(cfg.ctx_range[0], cfg.ctx_range[1] + 1, (S,), generator=g, dtype=torch.int64)
+    ql = torch.randint(cfg.q_range[0], cfg.q_range[1] + 1, (S,), generator=g, dtype=torch.int64)
+    if ctx_lens is not None:
+        ctx = torch.as_tensor(ctx_lens, dtype=torch.int64).clone()
+    if q_lens is not None:
+        ql = torch.as_tensor(q_lens, dtype=torch.int64).clone()
+    lens = ctx + ql
+    pages = (lens + ps - 1) // ps
+    width = max(1, int(pages.max().item()) if S else 1)
+    num_pages = int(pages.sum().item()) + spare_pages
+    perm = torch.randperm(num_pages, generator=g)
+    table = torch.full((S, width), -1, dtype=torch.int32)
+    off = 0
+    for s in range(S):
+        n = int(pages[s])
+        table[s, :n] = perm[off:off + n].to(torch.int32)
+        off += n
+    total_q = int(ql.sum().item())
+    cu = torch.zeros(S + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(ql, 0).to(torch.int32)
+    q = torch.randn(total_q, cfg.Hq, cfg.d, generator=g, dtype=torch.float32)
+    k_new = torch.randn(total_q, cfg.Hkv, cfg.d, generator=g, dtype=torch.float32)
+    v_new = torch.randn(total_q, cfg.Hkv, cfg.d, generator=g, dtype=torch.float32)
+    k_pool = torch.randn(num_pages, ps, cfg.Hkv, cfg.d, generator=g, dtype=torch.float32)
+    v_pool = torch.randn(num_pages, ps, cfg.Hkv, cfg.d, generator=g, dtype=torch.float32)
+    q, k_new, v_new, k_pool, v_pool = (t.to(torch.bfloat16) for t in (q, k_new, v_new, k_pool, v_pool))
+    if poison:
+        for s in range(S):
+            n = int(pages[s])
+            for t in range(int(ctx[s]), n * ps):
+                pg = int(table[s, t // ps])
+                k_pool[pg, t % ps] = float("nan")
+                v_pool[pg, t % ps] = float("nan")
+    dev = torch.device(device)
+    return {
+        "q": q.contiguous().to(dev),
+        "k_new": k_new.contiguous().to(dev),
+        "v_new": v_new.contiguous().to(dev),
+        "k_pool": k_pool.contiguous().to(dev),
+        "v_pool": v_pool.contiguous().to(dev),
+        "block_table": table.contiguous().to(dev),
+        "cu_seqlens_q": cu.contiguous().to(dev),
+        "seq_lens": lens.to(torch.int32).contiguous().to(dev),
+        "ctx_lens": ctx,
+        "q_lens": ql,
+        "page_size": ps,
+        "num_pages": num_pages,
+        "max_pages": width,
+        "total_q": total_q,
+        "scale": cfg.scale,
+    }
+
+
+def chunked_flops(ctx_lens, q_lens, Hq: int, d: int, causal: bool = True) -> float:
+    """4*d per visible (query, key) pair: new query i of a sequence sees
+    ctx + i + 1 keys under the causal mask, ctx + q otherwise."""
+    total = 0
+    for c, q in zip(torch.as_tensor(ctx_lens).tolist(), torch.as_tensor(q_lens).tolist()):
+        total += q * c + q * (q + 1) // 2 if causal else q * (c + q)
+    return 4.0 * Hq * d * total
+
+
+def chunked_append_bytes(q_lens, Hkv: int, d: int) -> float:
+    """HBM bytes of the append: K and V of every new token read once and
+    written once (2 tensors x 2 directions x Hkv x d x 2 bytes), plus the
+    block-table entries and lengths it reads."""
+    n = float(torch.as_tensor(q_lens).sum().item())
+    return n * 2 * 2 * Hkv * d * 2
 
 
 def make_prefill_inputs(cfg: PrefillConfig, device: str | torch.device = "cpu"):

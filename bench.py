@@ -13,7 +13,8 @@ i.e. the time-weighted fraction of the measured B200 peaks the step reaches
 separate prefill TFLOP/s and decode GB/s are in the line too.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--workload default|causal_mha|causal_gqa|long_causal|long_window|paged_decode|small_decode]
+       [--workload default|causal_mha|causal_gqa|long_causal|long_window|paged_decode|small_decode|
+                   chunked_prefill]
        [--decode-graph]
 Under torchrun each rank runs its own batch (seed offset by rank), no
 collective on the data path; rank 0 prints one JSON line.
@@ -41,7 +42,8 @@ from attention_flashattention_fwd_04_b200 import workloads as W  # noqa: E402
 
 METRIC = "causal prefill TFLOP/s and paged-decode KV GB/s, as fraction of B200 peaks"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
-KERNEL_SOURCES = ("attn_api.cu", "prefill_sm100.cuh", "decode_sm100.cuh", "ptx.cuh", "tmem_ldst.cuh", "exp2_poly.cuh")
+KERNEL_SOURCES = ("attn_api.cu", "prefill_sm100.cuh", "decode_sm100.cuh", "paged_append.cuh", "ptx.cuh", "tmem_ldst.cuh",
+                  "exp2_poly.cuh")
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -170,6 +172,12 @@ class ClockSampler:
 
 PREFILL_WORKLOADS = ("default", "causal_mha", "causal_gqa", "long_causal", "long_window", "tiny")
 DECODE_WORKLOADS = ("default", "paged_decode", "small_decode")
+CHUNKED_WORKLOADS = ("chunked_prefill",)
+
+
+def chunked_label(c) -> str:
+    return (f"append + chunked prefill {c.num_seqs} seqs Hq={c.Hq} Hkv={c.Hkv} d={c.d} page={c.page_size} "
+            f"context {c.ctx_range[0]}..{c.ctx_range[1]} new {c.q_range[0]}..{c.q_range[1]}")
 
 
 def prefill_label(c) -> str:
@@ -187,6 +195,11 @@ class Step:
         self.device = device
         self.prefill_cfg = None
         self.decode_cfg = None
+        self.chunked_cfg = None
+        self.resident = {}  # device state that persists across steps (the paged cache of chunked prefill)
+        if workload in CHUNKED_WORKLOADS:
+            base = W.CHUNKED_CONFIGS[workload]
+            self.chunked_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
         if workload in PREFILL_WORKLOADS:
             name = "causal_mha" if workload == "default" else workload
             base = W.PREFILL_CONFIGS[name]
@@ -211,7 +224,19 @@ class Step:
             self.host.update(dq=inp["q"], k_pool=inp["k_pool"], v_pool=inp["v_pool"],
                              block_table=inp["block_table"], seq_lens=inp["seq_lens"])
             self.bytes = W.decode_kv_bytes(inp["seq_lens"], c.Hkv, c.d, c.Hq, c.page_size)
+        self.chunked_inp = None
+        if self.chunked_cfg is not None:
+            c = self.chunked_cfg
+            inp = W.make_chunked_inputs(c)
+            self.chunked_inp = inp
+            self.host.update(cq=inp["q"], k_new=inp["k_new"], v_new=inp["v_new"], cu_q=inp["cu_seqlens_q"],
+                             c_seq_lens=inp["seq_lens"], c_table=inp["block_table"])
+            self.resident.update(c_k_pool=inp["k_pool"], c_v_pool=inp["v_pool"])
+            self.flops = W.chunked_flops(inp["ctx_lens"], inp["q_lens"], c.Hq, c.d)
+            self.bytes = W.chunked_append_bytes(inp["q_lens"], c.Hkv, c.d)
         for name, t in self.host.items():
+            self.dev[name] = t.to(device)
+        for name, t in self.resident.items():
             self.dev[name] = t.to(device)
         self._alloc_outputs()
         self.graph = None
@@ -226,6 +251,10 @@ class Step:
             q = self.dev["q"]
             self.dev["o"] = torch.empty_like(q)
             self.dev["lse"] = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+        if self.chunked_cfg is not None:
+            q = self.dev["cq"]
+            self.dev["co"] = torch.empty_like(q)
+            self.dev["clse"] = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
         if self.decode_cfg is not None:
             c, inp = self.decode_cfg, self.decode_inp
             need = api.paged_attn_decode_workspace_bytes(c.num_seqs, c.Hq, c.d, inp["max_pages"], c.page_size)
@@ -234,7 +263,28 @@ class Step:
             self.dev["dlse"] = torch.empty((c.num_seqs, c.Hq), dtype=torch.float32, device=dev)
 
     def launches_per_step(self) -> int:
-        return (1 if self.prefill_cfg is not None else 0) + (2 if self.decode_cfg is not None else 0)
+        return ((1 if self.prefill_cfg is not None else 0) + (2 if self.decode_cfg is not None else 0) +
+                (2 if self.chunked_cfg is not None else 0))
+
+    def run_chunked(self, d=None, ev=None, one_call=False):
+        """Append the chunk to the paged cache, then attend (two launches)."""
+        d = d or self.dev
+        c = self.chunked_cfg
+        if one_call:
+            self.api.paged_prefill_append(d["cq"], d["k_new"], d["v_new"], d["c_k_pool"], d["c_v_pool"], d["c_table"],
+                                          d["cu_q"], d["c_seq_lens"], True, c.scale, out=d["co"], lse=d["clse"])
+            return
+        stream = torch.cuda.current_stream()
+        if ev is not None:
+            ev[0].record(stream)
+        self.api.paged_kv_append(d["k_new"], d["v_new"], d["c_k_pool"], d["c_v_pool"], d["c_table"], d["cu_q"],
+                                 d["c_seq_lens"])
+        if ev is not None:
+            ev[1].record(stream)
+        self.api.paged_prefill(d["cq"], d["c_k_pool"], d["c_v_pool"], d["c_table"], d["cu_q"], d["c_seq_lens"], True,
+                               c.scale, out=d["co"], lse=d["clse"])
+        if ev is not None:
+            ev[2].record(stream)
 
     def run_prefill(self, d=None):
         d = d or self.dev
@@ -264,6 +314,14 @@ def config_dict(step: Step, n_gpus: int):
         cfg["prefill"] = {"B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "N": c.N, "d": c.d, "causal": c.causal,
                           "window_left": c.window_left, "scale": c.scale, "seed": c.seed,
                           "value_scale": c.value_scale, "k_offset_sigma": c.k_offset_sigma, "flops": step.flops}
+    if step.chunked_cfg is not None:
+        c, inp = step.chunked_cfg, step.chunked_inp
+        parts.append(chunked_label(c))
+        cfg["chunked"] = {"num_seqs": c.num_seqs, "Hq": c.Hq, "Hkv": c.Hkv, "d": c.d, "page_size": c.page_size,
+                          "context_range": list(c.ctx_range), "new_range": list(c.q_range),
+                          "total_new_tokens": inp["total_q"], "total_context_tokens": int(inp["ctx_lens"].sum()),
+                          "num_pages": inp["num_pages"], "seed": c.seed, "flops": step.flops,
+                          "append_bytes": step.bytes, "causal": True}
     if step.decode_cfg is not None:
         c = step.decode_cfg
         L = step.decode_inp["seq_lens"]
@@ -294,12 +352,37 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
 
     import oracle
 
-    prefill_cfg, decode_cfg, host, decode_inp = step_cfgs
+    prefill_cfg, decode_cfg, host, decode_inp, chunked = step_cfgs
     flops = 0.0
     nbytes = 0.0
     done_heads = 0
     done_seqs = 0
+    done_chunks = 0
+    if chunked is not None:
+        c, inp = chunked
+        cu = inp["cu_seqlens_q"].numpy()
+        lens = inp["seq_lens"].numpy()
+        table = inp["block_table"].numpy()
+        bits = [inp[n].view(torch.int16).numpy() for n in ("k_pool", "v_pool", "k_new", "v_new")]
+        cq = inp["q"].float().numpy()
     t0 = time.perf_counter()
+    if chunked is not None:
+        # the append (pure indexing, on the raw bf16 bits), then the attention
+        # of whole sequences (or the last 128 rows of one) until the budget
+        kb, vb = oracle.paged_append(*bits, table, cu, lens, c.page_size)
+        nbytes += W.chunked_append_bytes(inp["q_lens"], c.Hkv, c.d)
+        kp = torch.from_numpy(kb).view(torch.bfloat16).float().numpy()
+        vp = torch.from_numpy(vb).view(torch.bfloat16).float().numpy()
+        for s in range(c.num_seqs):
+            ql = int(cu[s + 1] - cu[s])
+            rows = min(ql, 128) if per_call else ql
+            ctx = int(lens[s]) - rows
+            oracle.paged_prefill(cq[cu[s + 1] - rows:cu[s + 1]], kp, vp, table[s:s + 1], np.array([0, rows]),
+                                 lens[s:s + 1], c.page_size, c.scale, True)
+            flops += W.chunked_flops([ctx], [rows], c.Hq, c.d)
+            done_chunks += 1
+            if time.perf_counter() - t0 > budget_s or per_call:
+                break
     if prefill_cfg is not None:
         c = prefill_cfg
         q, k, v = (host[n].float().numpy() for n in ("q", "k", "v"))
@@ -342,6 +425,9 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
         desc.append(f"{done_heads} prefill heads ({'last 128 rows' if per_call else 'all rows'})")
     if decode_cfg is not None:
         desc.append(f"{done_seqs} decode sequences")
+    if chunked is not None:
+        desc.append(f"append of all chunks + attention of {done_chunks} "
+                    f"{'chunk tails (last 128 rows)' if per_call else 'whole chunks'}")
     return {"flops": flops, "bytes": nbytes}, seconds, ", ".join(desc)
 
 
@@ -364,7 +450,7 @@ def run_reference(args, world, rank):
         return None
     peaks = load_peaks()
     step = StepHost(args.workload)
-    cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp)
+    cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp, step.chunked)
     for _ in range(args.warmup):
         oracle_sample(cfgs, 0.0, per_call=True)
     work_f = work_b = secs = 0.0
@@ -395,7 +481,12 @@ class StepHost:
         self.prefill_cfg = self.decode_cfg = None
         self.host = {}
         self.decode_inp = None
+        self.chunked = None
         parts = []
+        if workload in CHUNKED_WORKLOADS:
+            c = W.CHUNKED_CONFIGS[workload]
+            self.chunked = (c, W.make_chunked_inputs(c))
+            parts.append(chunked_label(c))
         if workload in PREFILL_WORKLOADS:
             name = "causal_mha" if workload == "default" else workload
             self.prefill_cfg = W.PREFILL_CONFIGS[name]
@@ -442,6 +533,8 @@ def run_ours(args, world, rank, local_rank):
             step.run_decode()
             if ev is not None:
                 ev[2].record(stream)
+        if step.chunked_cfg is not None:
+            step.run_chunked(ev=ev)
         if flush is not None:
             flush.fill_(1)
 
@@ -468,17 +561,20 @@ def run_ours(args, world, rank, local_rank):
     if api.device_status() != 0:
         raise RuntimeError("a kernel reported a device error in the timed region")
     total_s = start.elapsed_time(end) / 1e3
-    t_prefill = t_decode = 0.0
+    t_prefill = t_decode = t_append = t_cprefill = 0.0
     for i in range(args.steps):
         if step.prefill_cfg is not None:
             t_prefill += evs[i][0].elapsed_time(evs[i][1]) / 1e3
         if step.decode_cfg is not None:
             a = evs[i][1] if step.prefill_cfg is not None else (evs[i - 1][2] if i > 0 else start)
             t_decode += a.elapsed_time(evs[i][2]) / 1e3
+        if step.chunked_cfg is not None:
+            t_append += evs[i][0].elapsed_time(evs[i][1]) / 1e3
+            t_cprefill += evs[i][1].elapsed_time(evs[i][2]) / 1e3
     if flush is not None:
         # The L2 flush between steps is not work of the step: time the steps'
         # own event-bracketed regions (each one starts with a cold L2).
-        total_s = t_prefill
+        total_s = t_prefill + t_append + t_cprefill
     t_max = max_over_ranks(total_s, world, device)
     ideal_sum = sum_over_ranks(step.ideal_seconds(peaks) * args.steps, world, device)
     value = ideal_sum / t_max
@@ -510,11 +606,25 @@ def run_ours(args, world, rank, local_rank):
                                              "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                                              "us_per_launch": per * 1e6, "algorithmic": step.bytes}
         line["decode_kv_gbs"] = gbs
+    if step.chunked_cfg is not None:
+        per = t_append / args.steps
+        gbs = step.bytes / per / 1e9
+        kernels["paged_append_kernel"] = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                          "frac": gbs / peaks["hbm_gbs"], "us_per_launch": per * 1e6,
+                                          "algorithmic": step.bytes}
+        per = t_cprefill / args.steps
+        tfl = step.flops / per / 1e12
+        kernels["prefill_fwd_kernel (paged)"] = {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"],
+                                                 "unit": "TFLOP/s", "frac": tfl / peaks["bf16_tflops"],
+                                                 "us_per_launch": per * 1e6, "algorithmic": step.flops}
+        line["prefill_tflops"] = tfl
+        line["append_gbs"] = gbs
     dominant = max(kernels, key=lambda k: kernels[k]["us_per_launch"])
     traffic = load_traffic()
     dk = kernels[dominant]
     if dominant.startswith("prefill"):
-        tr = traffic.get(("prefill_fwd_kernel", step.prefill_cfg.name))
+        cfg_name = (step.prefill_cfg or step.chunked_cfg).name
+        tr = traffic.get(("prefill_fwd_kernel", cfg_name))
     else:
         parts = [traffic.get((k, step.decode_cfg.name)) for k in ("decode_split_kernel", "decode_merge_kernel")]
         tr = None if any(x is None for x in parts) else sum(parts)
@@ -524,8 +634,9 @@ def run_ours(args, world, rank, local_rank):
     line["kernels"] = kernels
     line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        chunked = (step.chunked_cfg, step.chunked_inp) if step.chunked_cfg is not None else None
         w, secs, desc = oracle_sample((step.prefill_cfg, step.decode_cfg, step.host,
-                                       getattr(step, "decode_inp", None)), args.cpu_seconds)
+                                       getattr(step, "decode_inp", None), chunked), args.cpu_seconds)
         ideal = w["flops"] / (peaks["bf16_tflops"] * 1e12) + w["bytes"] / (peaks["hbm_gbs"] * 1e9)
         cpu = {"value": ideal / secs, "unit": unit_string(), "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{desc}; {secs:.1f} s"}
@@ -542,7 +653,7 @@ def run_e2e(step: Step, args, world, device, peaks):
     inputs from pinned host memory and reads the results back."""
     pinned = {n: t.pin_memory() for n, t in step.host.items()}
     outs = {}
-    for n in ("o", "lse", "do", "dlse"):
+    for n in ("o", "lse", "do", "dlse", "co", "clse"):
         if n in step.dev:
             outs[n] = torch.empty(step.dev[n].shape, dtype=step.dev[n].dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
@@ -557,6 +668,8 @@ def run_e2e(step: Step, args, world, device, peaks):
             step.run_prefill()
         if step.decode_cfg is not None:
             step.run_decode()
+        if step.chunked_cfg is not None:
+            step.run_chunked(one_call=True)
         for n, t in outs.items():
             t.copy_(step.dev[n], non_blocking=True)
 
@@ -585,7 +698,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="default",
-                    choices=sorted(set(PREFILL_WORKLOADS) | set(DECODE_WORKLOADS)))
+                    choices=sorted(set(PREFILL_WORKLOADS) | set(DECODE_WORKLOADS) | set(CHUNKED_WORKLOADS)))
     ap.add_argument("--decode-graph", action="store_true",
                     help="run the decode step as a captured CUDA graph (split pass + merge)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

@@ -223,6 +223,64 @@ int paged_attn_decode_graph_launch(attn_decode_graph* graph, void* stream);
 int paged_attn_decode_graph_destroy(attn_decode_graph* graph);
 
 /*
+ * Appending to a paged cache, and chunked (paged) prefill.
+ *
+ * A step hands each sequence s a chunk of q_len(s) new tokens, packed by
+ * sequence: rows cu_seqlens_q[s] .. cu_seqlens_q[s+1]-1 of q [total_q, Hq, d]
+ * and of k_new / v_new [total_q, Hkv, d] (cu_seqlens_q [num_seqs+1] int32,
+ * non-decreasing, cu_seqlens_q[0] = 0, cu_seqlens_q[num_seqs] <= total_q).
+ * seq_lens [num_seqs] int32 is each sequence's length AFTER the step, so the
+ * chunk is logical tokens ctx .. seq_len-1 with ctx = seq_len - q_len, and
+ * the pools, block table, page_size, max_pages and num_pages are as for
+ * paged_attn_decode (pages for all seq_len tokens already assigned in the
+ * table: "blocks can be allocated on demand", "Fast Attention Kernels and
+ * Operator Fusion", section "Paged Attention Kernels").  page_size must be
+ * 16, 32, 64, 128 or 256.  A sequence whose lengths are out of range, or a
+ * table entry outside the pool, is skipped and reported through
+ * attn_device_status (bit 12); nothing is written outside the outputs and the
+ * pool slots of valid chunks.
+ *
+ * paged_kv_append -- writes new token i of sequence s (its K and V rows, all
+ * Hkv heads) to physical page block_table[s][(ctx + i) / page_size], slot
+ * (ctx + i) % page_size: the cache update the same page lists among the
+ * fusions of a layer (section "Operator Fusion").  Exact copies.  Every other
+ * pool slot is left as it was.
+ */
+int paged_kv_append(const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_pool, attn_bf16* v_pool,
+                    const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table,
+                    int num_seqs, int total_q, int Hkv, int d, int page_size, int max_pages, int num_pages,
+                    void* stream);
+
+/*
+ * paged_prefill -- attention of every sequence's new queries over its whole
+ * paged cache (the chunk included, so call it after paged_kv_append, or use
+ * paged_prefill_append).  New query i of sequence s is token ctx + i: with
+ * causal = 1 it sees keys 0 .. ctx + i, with causal = 0 all seq_len keys.
+ *   o    [total_q, Hq, d] bf16 (written: rows of valid chunks)
+ *   lse  [total_q, Hq] float32, natural log (written likewise)
+ * The same fused kernel as attn_fwd (scores stay on chip), with K/V read
+ * through the block table one page at a time; slots past a sequence's end
+ * are never used, whatever they hold.  d in {64, 128}, Hq % Hkv == 0,
+ * num_seqs <= 1024 (ATTN_ERR_UNSUPPORTED above that).  No workspace.
+ */
+int paged_prefill(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
+                  const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table, attn_bf16* o,
+                  float* lse, int num_seqs, int total_q, int Hq, int Hkv, int d, int page_size, int max_pages,
+                  int num_pages, int causal, float scale, void* stream);
+
+/*
+ * paged_prefill_append -- paged_kv_append followed by paged_prefill on the
+ * same stream, one call: the chunk's keys and values go into their pages and
+ * the attention then reads everything, the chunk included, through the table.
+ * All arguments are checked before either kernel is enqueued.
+ */
+int paged_prefill_append(const attn_bf16* q, const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_pool,
+                         attn_bf16* v_pool, const int32_t* cu_seqlens_q, const int32_t* seq_lens,
+                         const int32_t* block_table, attn_bf16* o, float* lse, int num_seqs, int total_q, int Hq,
+                         int Hkv, int d, int page_size, int max_pages, int num_pages, int causal, float scale,
+                         void* stream);
+
+/*
  * attn_device_status -- synchronises `stream`, then reads and clears the
  * device error word of the current device.  Returns ATTN_OK if no kernel
  * recorded an error since the last call, ATTN_ERR_DEVICE otherwise (the raw

@@ -124,3 +124,50 @@ def test_decode_graph_rejects_bad_arguments_on_the_host(lib):
     assert lib.paged_attn_decode_graph_create(*bad, ctypes.byref(h)) == 4
     assert lib.paged_attn_decode_graph_launch(None, None) == 1
     assert lib.paged_attn_decode_graph_destroy(None) == 0
+
+
+def _app(lib, kn=FAKE, vn=FAKE, kp=FAKE, vp=FAKE, cu=FAKE, sl=FAKE, bt=FAKE, S=2, total_q=5, Hkv=2, d=128,
+         ps=16, max_pages=4, num_pages=8):
+    return lib.paged_kv_append(kn, vn, kp, vp, cu, sl, bt, S, total_q, Hkv, d, ps, max_pages, num_pages, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(kn=None), 1), (dict(vn=None), 1), (dict(kp=None), 1), (dict(vp=None), 1), (dict(cu=None), 1),
+    (dict(sl=None), 1), (dict(bt=None), 1),
+    (dict(S=0), 2), (dict(total_q=-1), 2), (dict(Hkv=0), 2), (dict(d=96), 2), (dict(max_pages=0), 2),
+    (dict(num_pages=0), 2), (dict(ps=0), 2), (dict(num_pages=1 << 28, ps=16), 2),
+    (dict(ps=8), 5), (dict(ps=48), 5), (dict(ps=512), 5),
+    (dict(kn=FAKE + 8), 3), (dict(kp=FAKE + 2), 3), (dict(cu=FAKE + 2), 3), (dict(bt=FAKE + 1), 3),
+])
+def test_paged_kv_append_rejects(lib, kw, code):
+    assert _app(lib, **kw) == code
+
+
+def test_paged_kv_append_with_no_new_tokens_is_a_no_op(lib):
+    # nothing to copy: no kernel is launched, the new-row pointers are not needed
+    assert _app(lib, kn=None, vn=None, total_q=0) == 0
+
+
+def _pp(lib, q=FAKE, kp=FAKE, vp=FAKE, cu=FAKE, sl=FAKE, bt=FAKE, o=FAKE, lse=FAKE, S=2, total_q=5, Hq=8, Hkv=2,
+        d=128, ps=16, max_pages=4, num_pages=8, causal=1, scale=0.1, fn="paged_prefill"):
+    if fn == "paged_prefill":
+        return lib.paged_prefill(q, kp, vp, cu, sl, bt, o, lse, S, total_q, Hq, Hkv, d, ps, max_pages, num_pages,
+                                 causal, scale, None)
+    return lib.paged_prefill_append(q, FAKE, FAKE, kp, vp, cu, sl, bt, o, lse, S, total_q, Hq, Hkv, d, ps,
+                                    max_pages, num_pages, causal, scale, None)
+
+
+@pytest.mark.parametrize("fn", ["paged_prefill", "paged_prefill_append"])
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(lse=None), 1), (dict(kp=None), 1), (dict(bt=None), 1),
+    (dict(S=0), 2), (dict(Hq=0), 2), (dict(Hq=6, Hkv=4), 2), (dict(d=80), 2), (dict(causal=2), 2),
+    (dict(scale=0.0), 2), (dict(scale=float("nan")), 2), (dict(total_q=1 << 30, Hq=8), 2),
+    (dict(ps=24), 5), (dict(S=1025), 5),
+    (dict(q=FAKE + 8), 3), (dict(o=FAKE + 4), 3), (dict(lse=FAKE + 2), 3), (dict(sl=FAKE + 2), 3),
+])
+def test_paged_prefill_rejects(lib, fn, kw, code):
+    assert _pp(lib, fn=fn, **kw) == code
+
+
+def test_paged_prefill_with_no_new_tokens_is_a_no_op(lib):
+    assert _pp(lib, total_q=0) == 0
