@@ -516,6 +516,8 @@ int validate_paged_prefill(const attn_bf16* q, const attn_bf16* k_pool, const at
   if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_SHAPE;
   if (static_cast<long long>(total_q) * Hq > INT_MAX) return ATTN_ERR_SHAPE;
   if (num_seqs > attn::kPagedMaxSeqs) return ATTN_ERR_UNSUPPORTED;
+  // Query blocks of 256 rows: at most ceil(q_len / 256) per sequence.
+  if ((static_cast<long long>(total_q) + 255LL * num_seqs) / 256 > attn::kPagedMaxBlocks) return ATTN_ERR_UNSUPPORTED;
   if (misaligned16(q) || misaligned16(o) || misaligned4(lse)) return ATTN_ERR_ALIGN;
   return ATTN_OK;
 }

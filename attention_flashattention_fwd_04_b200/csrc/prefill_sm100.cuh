@@ -80,7 +80,8 @@ struct PrefillParams {
   int page_box;                // rows per K/V TMA box: min(page_size, 128)
 };
 
-constexpr int kPagedMaxSeqs = 1024;  // sequences per paged-prefill call
+constexpr int kPagedMaxSeqs = 1024;    // sequences per paged-prefill call
+constexpr int kPagedMaxBlocks = 2048;  // 256-row query blocks per paged-prefill call
 
 constexpr int kPrefillThreads = 512;
 constexpr float kRescaleThreshold = 8.0f;  // in log2 units
@@ -97,10 +98,11 @@ struct PrefillLayout {
   static constexpr int kV = kK + NS * kTileBytes;
   static constexpr int kStats = kV + NS * kTileBytes;  // float [tile 2][slot 2][m,l][128 rows]
   static constexpr int kStatsBytes = 2 * 2 * 2 * 128 * 4;
-  // Paged: per-sequence table cached at kernel start: item offsets [S+1],
-  // cu_q [S+1], seq_lens [S], and 16 ints of scan scratch.
+  // Paged: cached at kernel start: the query blocks in processing order
+  // [kPagedMaxBlocks], cu_q [S+1], seq_lens [S], the block count and 16 ints
+  // of scan scratch.
   static constexpr int kSeq = kStats + kStatsBytes;
-  static constexpr int kSeqBytes = PAGED ? (3 * kPagedMaxSeqs + 2 + 16) * 4 : 0;
+  static constexpr int kSeqBytes = PAGED ? (kPagedMaxBlocks + 2 * kPagedMaxSeqs + 1 + 1 + 16) * 4 : 0;
   static constexpr int kBar = (kSeq + kSeqBytes + 7) / 8 * 8;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarQEmpty = 1;
@@ -141,30 +143,35 @@ struct PrefillItem {
 
 // Sequence table of the paged kernels, in shared memory.
 struct PagedSeqs {
-  const int* item_off;  // [S + 1]: first item of each sequence, item_off[S] = total
-  const int* cu_q;      // [S + 1]
-  const int* lens;      // [S]
+  const int* blocks;   // [num_blocks]: query block (sequence s, block m) as s * 2048 + m, heaviest first
+  const int* cu_q;     // [S + 1]
+  const int* lens;     // [S]
+  const int* nblocks;  // number of query blocks
 };
 
+// KV tiles the two query tiles of block m of a chunk visit (its work).
+template <bool CAUSAL>
+__device__ __forceinline__ int paged_block_tiles(int pos0, int n_q, int n_kv, int m) {
+  const int last0 = CAUSAL ? min(pos0 + m * 256 + 127, n_kv - 1) : n_kv - 1;
+  const int last1 = CAUSAL ? min(pos0 + m * 256 + 255, n_kv - 1) : n_kv - 1;
+  return last0 / 128 + 1 + (m * 256 + 128 < n_q ? last1 / 128 + 1 : 0);
+}
+
+// Item idx = (block rank idx / Hq, head idx % Hq).
 template <bool CAUSAL>
 __device__ __forceinline__ bool paged_item(int idx, const PrefillParams& p, const PagedSeqs& sq,
                                            PrefillItem& it) {
-  if (idx >= sq.item_off[p.num_seqs]) return false;
-  int lo = 0, hi = p.num_seqs;  // item_off[lo] <= idx < item_off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (sq.item_off[mid] <= idx) lo = mid; else hi = mid;
-  }
-  const int local = idx - sq.item_off[lo];
-  it.b = lo;
-  it.q0 = sq.cu_q[lo];
-  it.n_q = sq.cu_q[lo + 1] - it.q0;
-  it.n_kv = sq.lens[lo];
+  const int rank = idx / p.Hq;
+  if (rank >= *sq.nblocks) return false;
+  const int blk = sq.blocks[rank];
+  const int s = blk >> 11;
+  it.b = s;
+  it.m = blk & 2047;
+  it.h = idx - rank * p.Hq;
+  it.q0 = sq.cu_q[s];
+  it.n_q = sq.cu_q[s + 1] - it.q0;
+  it.n_kv = sq.lens[s];
   it.pos0 = it.n_kv - it.n_q;
-  const int n_m = (it.n_q + 255) / 256;
-  it.h = local % p.Hq;
-  const int rank = local / p.Hq;  // 0 = heaviest (causal)
-  it.m = CAUSAL ? (n_m - 1 - rank) : rank;
   {
     const int r0 = it.pos0 + it.m * 256;
     const int last_key = CAUSAL ? min(r0 + 127, it.n_kv - 1) : it.n_kv - 1;
@@ -224,30 +231,38 @@ __device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, 
 }
 
 // Paged kernels: every CTA caches the sequence table in shared memory and
-// counts the work items of each sequence (ceil(q_len / 256) query blocks per
-// head) with a block-wide prefix sum.  A sequence whose lengths are out of
-// range gets no items and sets kErrPagedTable.  Called by all threads.
-__device__ __forceinline__ void paged_seq_table(const PrefillParams& p, int* off, int* cuq, int* lens,
-                                                int* scratch) {
+// lists the 256-row query blocks of all chunks, heaviest (most KV tiles)
+// first, so the persistent CTAs, dealt items in that order, finish together.
+// A sequence whose lengths are out of range gets no blocks and sets
+// kErrPagedTable.  `scratch` is shared memory that is free until the main
+// loop (the V ring): 2048 sort keys and S + 1 block offsets.  Called by all
+// threads; ends with a barrier.
+template <bool CAUSAL>
+__device__ __forceinline__ void paged_seq_table(const PrefillParams& p, int* blocks, int* cuq, int* lens,
+                                                int* nblocks, int* wsum, uint8_t* scratch) {
   const int S = p.num_seqs;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int nw = static_cast<int>(blockDim.x >> 5);
+  const int tid = static_cast<int>(threadIdx.x);
+  const int nthreads = static_cast<int>(blockDim.x);
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int nw = nthreads >> 5;
+  uint64_t* keys = reinterpret_cast<uint64_t*>(scratch);
+  int* boff = reinterpret_cast<int*>(scratch + kPagedMaxBlocks * 8);  // [S + 1] first block of each sequence
   int v[2];
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
-    const int s = 2 * static_cast<int>(threadIdx.x) + e;
+    const int sq = 2 * tid + e;
     v[e] = 0;
-    if (s < S) {
-      const int a = p.cu_q[s], b = p.cu_q[s + 1], len = p.seq_lens[s];
-      cuq[s] = a;
-      lens[s] = len;
-      if (s == S - 1) cuq[S] = b;
+    if (sq < S) {
+      const int a = p.cu_q[sq], b = p.cu_q[sq + 1], len = p.seq_lens[sq];
+      cuq[sq] = a;
+      lens[sq] = len;
+      if (sq == S - 1) cuq[S] = b;
       const int nq = b - a;
       if (a < 0 || nq < 0 || b > p.total_q || nq > len || len > p.max_pages * p.page_size) {
         if (blockIdx.x == 0) atomicOr(&g_attn_device_error, kErrPagedTable);
       } else {
-        v[e] = (nq + 255) / 256 * p.Hq;
+        v[e] = (nq + 255) / 256;
       }
     }
   }
@@ -258,23 +273,70 @@ __device__ __forceinline__ void paged_seq_table(const PrefillParams& p, int* off
     const int y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) scratch[warp] = x;
+  if (lane == 31) wsum[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = lane < nw ? scratch[lane] : 0;
+    int w = lane < nw ? wsum[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    if (lane < nw) scratch[lane] = w;
+    if (lane < nw) wsum[lane] = w;
   }
   __syncthreads();
-  const int before = x - tot + (warp > 0 ? scratch[warp - 1] : 0);
-  const int s0 = 2 * static_cast<int>(threadIdx.x);
-  if (s0 < S) off[s0] = before;
-  if (s0 + 1 < S) off[s0 + 1] = before + v[0];
-  if (threadIdx.x == 0) off[S] = scratch[nw - 1];
+  const int before = x - tot + (warp > 0 ? wsum[warp - 1] : 0);
+  if (2 * tid < S) boff[2 * tid] = before;
+  if (2 * tid + 1 < S) boff[2 * tid + 1] = before + v[0];
+  int nb = wsum[nw - 1];
+  if (nb > kPagedMaxBlocks) {  // only with inconsistent offsets (the host bounds the sum)
+    if (blockIdx.x == 0 && tid == 0) atomicOr(&g_attn_device_error, kErrPagedTable);
+    nb = 0;
+  }
+  if (tid == 0) {
+    boff[S] = nb;
+    *nblocks = nb;
+  }
+  __syncthreads();
+  // Sort keys: work (KV tiles) high, then the block id s * 2048 + m inverted,
+  // so equal work keeps sequence order; padding keys are 0 and sort last.
+  int n = 1;
+  while (n < nb) n <<= 1;
+  for (int i = tid; i < n; i += nthreads) {
+    uint64_t key = 0;
+    if (i < nb) {
+      int lo = 0, hi = S;  // boff[lo] <= i < boff[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (boff[mid] <= i) lo = mid; else hi = mid;
+      }
+      const int m = i - boff[lo];
+      const int nq = cuq[lo + 1] - cuq[lo];
+      const int w = paged_block_tiles<CAUSAL>(lens[lo] - nq, nq, lens[lo], m);
+      key = (static_cast<uint64_t>(w) << 32) | (0xffffffffu - static_cast<uint32_t>(lo * 2048 + m));
+    }
+    keys[i] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= n; k <<= 1) {  // bitonic sort, descending
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < n; i += nthreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint64_t a = keys[i], b = keys[ixj];
+          if (((i & k) == 0) ? (a < b) : (a > b)) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = tid; i < nb; i += nthreads)
+    blocks[i] = static_cast<int>(0xffffffffu - static_cast<uint32_t>(keys[i] & 0xffffffffu));
+  fence_proxy_async_smem();  // TMA (async proxy) will overwrite the scratch keys
+  __syncthreads();
 }
 
 // Register split per warpgroup (launch: 512 threads x 128 registers):
@@ -311,11 +373,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
   PagedSeqs sq{};
   if constexpr (PAGED) {
-    int* off = reinterpret_cast<int*>(smem + L::kSeq);
-    int* cuq = off + kPagedMaxSeqs + 1;
+    int* blocks = reinterpret_cast<int*>(smem + L::kSeq);
+    int* cuq = blocks + kPagedMaxBlocks;
     int* lens = cuq + kPagedMaxSeqs + 1;
-    paged_seq_table(p, off, cuq, lens, lens + kPagedMaxSeqs);
-    sq = PagedSeqs{off, cuq, lens};
+    int* nblocks = lens + kPagedMaxSeqs;
+    paged_seq_table<CAUSAL>(p, blocks, cuq, lens, nblocks, nblocks + 1, smem + L::kV);
+    sq = PagedSeqs{blocks, cuq, lens, nblocks};
   }
 
   if (threadIdx.x == 0) {
@@ -363,6 +426,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int kv_it = 0, k_issued = 0, v_issued = 0, q_issued = 0;
       bool ok = true;
       PrefillItem it{};
+      // Paged: the tile whose pages t_row / t_valid describe (lane b: box b),
+      // and a 32-entry window of the item's block-table row (lane l: entry
+      // win_base + l) with the next 32 entries prefetched in win_next.
+      int tile_j = -1, t_row = 0, t_valid = 0;
+      int win_base = -(1 << 30), win_page = -1, win_next = -1;
+      bool have_next = false;
       auto wait0 = [&](uint32_t b, uint32_t parity, unsigned int code) -> bool {
         int r = 1;
         if (lane == 0) r = mbar_wait(b, parity, code) ? 1 : 0;
@@ -381,22 +450,39 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           // Box b (lane b) holds keys 128j + b*pb ...: a page (or a 128-key
           // part of one) found through the block table.  Boxes wholly past the
           // sequence start outside the pool, so TMA fills them with zeros.
+          // K and V of a tile share their pages: resolved once, for K.
           const int pb = p.page_box;
           const int nbox = 128 / pb;
-          int row = p.num_pages * p.page_size;
-          int valid = pb;  // rows of the box inside the sequence
-          if (lane < nbox) {
+          if (tile_j != j) {
+            tile_j = j;
+            const int lp_first = (j * 128) / p.page_size;
+            const int lp_last = (j * 128 + 127) / p.page_size;
+            if (lp_first < win_base || lp_last >= win_base + 32) {
+              // Lane l holds the table entry of logical page win_base + l; the
+              // next 32 entries are fetched ahead, while this window is used.
+              const int* trow = p.block_table + static_cast<size_t>(it.b) * p.max_pages;
+              const bool follow = have_next && lp_first == win_base + 32;
+              win_base = lp_first;
+              win_page = follow ? win_next : (win_base + lane < p.max_pages ? trow[win_base + lane] : -1);
+              win_next = win_base + 32 + lane < p.max_pages ? trow[win_base + 32 + lane] : -1;
+              have_next = true;
+            }
             const int pos = j * 128 + lane * pb;
-            if (pos < it.n_kv) {
-              int pg = p.block_table[static_cast<size_t>(it.b) * p.max_pages + pos / p.page_size];
+            const int pg_raw = __shfl_sync(0xffffffffu, win_page, (pos / p.page_size - win_base) & 31);
+            t_row = p.num_pages * p.page_size;
+            t_valid = pb;
+            if (lane < nbox && pos < it.n_kv) {
+              int pg = pg_raw;
               if (pg < 0 || pg >= p.num_pages) {
                 atomicOr(&g_attn_device_error, kErrPagedTable);
                 pg = 0;  // keep every copy inside the pool; the result is flagged invalid
               }
-              row = pg * p.page_size + pos % p.page_size;
-              valid = min(pb, it.n_kv - pos);
+              t_row = pg * p.page_size + pos % p.page_size;
+              t_valid = min(pb, it.n_kv - pos);
             }
           }
+          const int row = t_row;
+          const int valid = t_valid;
           // The box with the sequence's last token, when only part of it is
           // used, comes through plain loads: the slots past the end may hold
           // anything (even NaN), so they are written as zeros instead.
@@ -428,13 +514,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             else
               mbar_arrive(full);
           }
-          for (int b = 0; b < nbox; ++b) {
-            const int rb = __shfl_sync(0xffffffffu, row, b);
-            if (lane == 0 && ((part >> b) & 1u) == 0u)
-              for (int c = 0; c < D / 64; ++c)
-                tma_load_3d(dst + static_cast<uint32_t>(c * L::kBoxBytes + b * pb * 128), map, full, c * 64, rb,
-                            kz);
-          }
+          // Lane b issues box b: a one-thread loop over the boxes (a shuffle
+          // and two copies each) made the producer the bottleneck for
+          // 16-token pages.
+          __syncwarp();
+          if (lane < nbox && ((part >> lane) & 1u) == 0u)
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(dst + static_cast<uint32_t>(c * L::kBoxBytes + lane * pb * 128), map, full, c * 64, row,
+                          kz);
         }
       };
       auto load_k = [&](int j, int kz) -> bool {
@@ -459,6 +546,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int qrow = (PAGED ? it.q0 : 0) + it.m * 256;
         // GQA: consecutive query heads share a KV head
         const int kz = (PAGED ? 0 : it.b * p.Hkv) + it.h / p.group;
+        tile_j = -1;  // a new item: its own sequence, pages and table row
+        win_base = -(1 << 30);
+        have_next = false;
         // The item's first K tile first: it can land while the previous item
         // still holds Q.
         if (!(ok = load_k(it.jb, kz))) break;

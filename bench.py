@@ -625,6 +625,8 @@ def run_ours(args, world, rank, local_rank):
     if dominant.startswith("prefill"):
         cfg_name = (step.prefill_cfg or step.chunked_cfg).name
         tr = traffic.get(("prefill_fwd_kernel", cfg_name))
+    elif dominant == "paged_append_kernel":
+        tr = traffic.get(("paged_append_kernel", step.chunked_cfg.name))
     else:
         parts = [traffic.get((k, step.decode_cfg.name)) for k in ("decode_split_kernel", "decode_merge_kernel")]
         tr = None if any(x is None for x in parts) else sum(parts)

@@ -261,7 +261,8 @@ int paged_kv_append(const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k
  * The same fused kernel as attn_fwd (scores stay on chip), with K/V read
  * through the block table one page at a time; slots past a sequence's end
  * are never used, whatever they hold.  d in {64, 128}, Hq % Hkv == 0,
- * num_seqs <= 1024 (ATTN_ERR_UNSUPPORTED above that).  No workspace.
+ * num_seqs <= 1024 and (total_q + 255 * num_seqs) / 256 <= 2048 (at most 2048
+ * query blocks of 256 rows; ATTN_ERR_UNSUPPORTED beyond).  No workspace.
  */
 int paged_prefill(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool,
                   const int32_t* cu_seqlens_q, const int32_t* seq_lens, const int32_t* block_table, attn_bf16* o,

@@ -162,7 +162,7 @@ def _pp(lib, q=FAKE, kp=FAKE, vp=FAKE, cu=FAKE, sl=FAKE, bt=FAKE, o=FAKE, lse=FA
     (dict(q=None), 1), (dict(o=None), 1), (dict(lse=None), 1), (dict(kp=None), 1), (dict(bt=None), 1),
     (dict(S=0), 2), (dict(Hq=0), 2), (dict(Hq=6, Hkv=4), 2), (dict(d=80), 2), (dict(causal=2), 2),
     (dict(scale=0.0), 2), (dict(scale=float("nan")), 2), (dict(total_q=1 << 30, Hq=8), 2),
-    (dict(ps=24), 5), (dict(S=1025), 5),
+    (dict(ps=24), 5), (dict(S=1025), 5), (dict(total_q=600000, Hq=2, Hkv=2), 5),
     (dict(q=FAKE + 8), 3), (dict(o=FAKE + 4), 3), (dict(lse=FAKE + 2), 3), (dict(sl=FAKE + 2), 3),
 ])
 def test_paged_prefill_rejects(lib, fn, kw, code):

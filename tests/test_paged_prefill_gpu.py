@@ -36,6 +36,13 @@ def to_cuda(inp):
             for k, v in inp.items()}
 
 
+def nan_outputs(g):
+    """Outputs pre-filled with NaN: a row the kernel skips cannot pass."""
+    o = torch.full_like(g["q"], float("nan"))
+    lse = torch.full(g["q"].shape[:2], float("nan"), device=g["q"].device)
+    return o, lse
+
+
 def oracle_append(inp):
     """Pools after the append, as raw bf16 bit patterns (pure indexing)."""
     kp, vp = oracle.paged_append(bits(inp["k_pool"]), bits(inp["v_pool"]), bits(inp["k_new"]), bits(inp["v_new"]),
@@ -82,8 +89,30 @@ def test_append_then_prefill_matches_the_oracle(S, Hq, Hkv, d, ps, ctx, ql, caus
     cfg = W.ChunkedConfig("t", S, Hq, Hkv, d, ps, (0, 1), (1, 1), seed=sum(ctx) + sum(ql) + ps)
     inp = W.make_chunked_inputs(cfg, poison=True, ctx_lens=ctx, q_lens=ql, spare_pages=3)
     g = to_cuda(inp)
-    o, lse = api.paged_prefill_append(g["q"], g["k_new"], g["v_new"], g["k_pool"], g["v_pool"], g["block_table"],
-                                      g["cu_seqlens_q"], g["seq_lens"], causal=causal, scale=inp["scale"])
+    o, lse = nan_outputs(g)
+    api.paged_prefill_append(g["q"], g["k_new"], g["v_new"], g["k_pool"], g["v_pool"], g["block_table"],
+                             g["cu_seqlens_q"], g["seq_lens"], causal=causal, scale=inp["scale"], out=o, lse=lse)
+    assert api.device_status() == 0
+    kp, vp = oracle_append(inp)
+    assert np.array_equal(bits(g["k_pool"]), kp) and np.array_equal(bits(g["v_pool"]), vp)
+    ro, rl = oracle_prefill(inp, kp, vp, causal)
+    assert_close(o, lse, ro, rl)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_many_sequences_with_empty_chunks(causal):
+    """300 sequences (blocks sorted by work on the device, 2 sequences per
+    thread in the scan), a third of them with no new tokens."""
+    S = 300
+    rng = np.random.default_rng(46)
+    ctx = rng.integers(0, 400, S).tolist()
+    ql = [0 if i % 3 == 0 else int(x) for i, x in enumerate(rng.integers(1, 300, S))]
+    cfg = W.ChunkedConfig("t", S, 4, 2, 64, 16, (0, 1), (1, 1), seed=46)
+    inp = W.make_chunked_inputs(cfg, poison=True, ctx_lens=ctx, q_lens=ql)
+    g = to_cuda(inp)
+    o, lse = nan_outputs(g)
+    api.paged_prefill_append(g["q"], g["k_new"], g["v_new"], g["k_pool"], g["v_pool"], g["block_table"],
+                             g["cu_seqlens_q"], g["seq_lens"], causal=causal, scale=inp["scale"], out=o, lse=lse)
     assert api.device_status() == 0
     kp, vp = oracle_append(inp)
     assert np.array_equal(bits(g["k_pool"]), kp) and np.array_equal(bits(g["v_pool"]), vp)
