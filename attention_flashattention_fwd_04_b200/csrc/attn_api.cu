@@ -475,8 +475,6 @@ int attn_device_status(void* stream, unsigned int* bits) {
 
 namespace {
 
-constexpr int kAppendBlocksPerSm = 16;
-
 bool page_size_supported(int page_size) {
   return page_size == 16 || page_size == 32 || page_size == 64 || page_size == 128 || page_size == 256;
 }
@@ -543,10 +541,9 @@ int launch_append(const attn_bf16* k_new, const attn_bf16* v_new, attn_bf16* k_p
   p.max_pages = max_pages;
   p.num_pages = num_pages;
   p.page_size = page_size;
-  constexpr int kWarps = attn::kAppendThreads / 32;  // one new token per warp
-  const long long want = (static_cast<long long>(total_q) + kWarps - 1) / kWarps;
-  const long long cap = static_cast<long long>(sms) * kAppendBlocksPerSm;
-  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+  // One warp per kAppendTokensPerWarp consecutive new tokens.
+  constexpr long long kTokensPerBlock = attn::kAppendThreads / 32 * attn::kAppendTokensPerWarp;
+  const unsigned grid = static_cast<unsigned>((static_cast<long long>(total_q) + kTokensPerBlock - 1) / kTokensPerBlock);
   attn::paged_append_kernel<<<grid, attn::kAppendThreads, 0, stream>>>(p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? ATTN_OK : fail_cuda(e);

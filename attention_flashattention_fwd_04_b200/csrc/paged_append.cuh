@@ -9,9 +9,12 @@
 // token ctx + i (ctx = seq_lens[s] - q_len), written to physical page
 // block_table[s][(ctx + i) / page_size], slot (ctx + i) % page_size.
 //
-// One warp per new token: its [Hkv, D] rows of K and of V are contiguous both
-// in the packed input and in the page slot, so each is one straight copy of
-// Hkv * D * 2 bytes in 16-byte vectors.  HBM-bound.
+// Each warp copies a run of consecutive new tokens: one binary search finds
+// the sequence of the first, the rest walk forward.  A token's [Hkv, D] rows
+// of K and of V are contiguous both in the packed input and in the page
+// slot, so each is one straight copy of Hkv * D * 2 bytes in 16-byte
+// vectors; all of a token's vectors are loaded before any is stored, so the
+// loads overlap.  HBM-bound.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,28 +33,39 @@ struct AppendParams {
 };
 
 constexpr int kAppendThreads = 256;
+constexpr int kAppendTokensPerWarp = 4;
+constexpr int kAppendVecsPerLane = 4;  // 16-byte vectors per lane and tensor in one batch
 
 __global__ void __launch_bounds__(kAppendThreads) paged_append_kernel(const AppendParams p) {
   const int lane = threadIdx.x & 31;
-  const int warps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+  const int gw = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int t_begin = gw * kAppendTokensPerWarp;
+  if (t_begin >= p.total_q) return;
+  const int t_end = min(p.total_q, t_begin + kAppendTokensPerWarp);
   const int vecs = p.Hkv * p.D / 8;  // 16-byte vectors per token and tensor
-  for (int t = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); t < p.total_q; t += warps) {
-    // Sequence of packed row t: the last s with cu_q[s] <= t.
-    int lo = 0, hi = p.num_seqs;
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (p.cu_q[mid] <= t) lo = mid; else hi = mid;
+  // Sequence of the first token: the last s with cu_q[s] <= t_begin.
+  int lo = 0, hi = p.num_seqs;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (p.cu_q[mid] <= t_begin) lo = mid; else hi = mid;
+  }
+  int s = lo;
+  int q0 = p.cu_q[s], q1 = p.cu_q[s + 1], len = p.seq_lens[s];
+  for (int t = t_begin; t < t_end; ++t) {
+    while (t >= q1 && s + 1 < p.num_seqs) {  // next non-empty sequence
+      ++s;
+      q0 = q1;
+      q1 = p.cu_q[s + 1];
+      len = p.seq_lens[s];
     }
-    const int q0 = p.cu_q[lo];
-    const int nq = p.cu_q[lo + 1] - q0;
-    const int len = p.seq_lens[lo];
+    const int nq = q1 - q0;
     const int i = t - q0;
     if (i < 0 || i >= nq || nq > len || len > p.max_pages * p.page_size) {
       if (lane == 0) atomicOr(&g_attn_device_error, kErrPagedTable);
       continue;
     }
     const int pos = len - nq + i;
-    const int pg = p.block_table[static_cast<size_t>(lo) * p.max_pages + pos / p.page_size];
+    const int pg = p.block_table[static_cast<size_t>(s) * p.max_pages + pos / p.page_size];
     if (pg < 0 || pg >= p.num_pages) {
       if (lane == 0) atomicOr(&g_attn_device_error, kErrPagedTable);
       continue;  // nothing is written outside the pool
@@ -62,11 +76,24 @@ __global__ void __launch_bounds__(kAppendThreads) paged_append_kernel(const Appe
     const uint4* vs = reinterpret_cast<const uint4*>(p.v_new) + src;
     uint4* kd = reinterpret_cast<uint4*>(p.k_pool) + dst;
     uint4* vd = reinterpret_cast<uint4*>(p.v_pool) + dst;
-    for (int x = lane; x < vecs; x += 32) {
-      const uint4 a = ks[x];
-      const uint4 b = vs[x];
-      kd[x] = a;
-      vd[x] = b;
+    for (int base = 0; base < vecs; base += 32 * kAppendVecsPerLane) {
+      uint4 a[kAppendVecsPerLane], b[kAppendVecsPerLane];
+#pragma unroll
+      for (int u = 0; u < kAppendVecsPerLane; ++u) {
+        const int x = base + u * 32 + lane;
+        if (x < vecs) {
+          a[u] = ks[x];
+          b[u] = vs[x];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kAppendVecsPerLane; ++u) {
+        const int x = base + u * 32 + lane;
+        if (x < vecs) {
+          kd[x] = a[u];
+          vd[x] = b[u];
+        }
+      }
     }
   }
 }

@@ -484,8 +484,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const int row = t_row;
           const int valid = t_valid;
           // The box with the sequence's last token, when only part of it is
-          // used, comes through plain loads: the slots past the end may hold
-          // anything (even NaN), so they are written as zeros instead.
+          // used, comes through 16-byte cp.async copies instead: the slots past
+          // the end may hold anything (even NaN), so they are filled with
+          // zeros (source size 0).  Each lane's copies hold the stage's phase
+          // open until they land.
           const unsigned part = __ballot_sync(0xffffffffu, lane < nbox && valid < pb);
           if (part != 0u) {
             const int b = __ffs(part) - 1;
@@ -497,14 +499,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               const int c = (idx % kChunks) / 8;   // 64-column half
               const int ch = idx % 8;              // chunk within the 128-byte row
               const int tr = b * pb + r;           // row within the tile
-              uint4 val = make_uint4(0u, 0u, 0u, 0u);
-              if (r < pval)
-                val = *reinterpret_cast<const uint4*>(
-                    pool + ((static_cast<size_t>(prow + r) * p.Hkv + kz) * D + c * 64 + ch * 8));
-              const uint32_t a = dst + static_cast<uint32_t>(c * L::kBoxBytes + tr * 128 + ((ch ^ (tr & 7)) << 4));
-              *reinterpret_cast<uint4*>(smem + (a - base)) = val;
+              const bool in = r < pval;
+              const __nv_bfloat16* src =
+                  in ? pool + ((static_cast<size_t>(prow + r) * p.Hkv + kz) * D + c * 64 + ch * 8) : pool;
+              cp_async_16(dst + static_cast<uint32_t>(c * L::kBoxBytes + tr * 128 + ((ch ^ (tr & 7)) << 4)), src,
+                          in ? 16u : 0u);
             }
-            fence_proxy_async_smem();
+            cp_async_mbar_arrive(full);
           }
           __syncwarp();
           const int ntma = nbox - (part != 0u ? 1 : 0);
