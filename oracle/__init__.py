@@ -6,9 +6,11 @@ reference legs may import this package.  The product path never does.
 
 from .attention import (  # noqa: F401
     attention_forward,
+    attention_forward_fp8,
     attention_head,
     attention_rows,
     attention_scores,
+    fp8_e4m3_decode,
     gather_paged_kv,
     gqa_kv_head,
     paged_append,

@@ -35,6 +35,11 @@ Readings where the pages are silent (each is restated where it is used):
   t % page_size ("Paged Attention Kernels" section and its block-table figure,
   logical blocks 0,1,2,3 -> physical 17,4,29,8).  Decode has one query per
   sequence that sees all seq_len cached keys.
+* FP8 inputs (the anylearn.cc lesson's FA v3 section: Q K^T and P V computed
+  in FP8): Q, K, V arrive as e4m3 codes with one descale factor per tensor;
+  the operation is attention over the decoded values times their descales
+  (e4m3: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals at
+  exponent field 0, no infinities, the all-ones code NaN).
 * appending to the cache / chunked prefill ("Operator Fusion" section: the
   KV cache is updated as keys and values are produced; "Paged Attention
   Kernels": blocks are allocated as the cache grows): a sequence holding
@@ -73,6 +78,8 @@ __all__ = [
     "paged_decode",
     "paged_append",
     "paged_prefill",
+    "fp8_e4m3_decode",
+    "attention_forward_fp8",
 ]
 
 
@@ -292,3 +299,30 @@ def paged_prefill(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens, page_s
             o[q0:q0 + q_len, h] = o_h
             lse[q0:q0 + q_len, h] = l_h
     return o, lse
+
+
+def fp8_e4m3_decode(codes) -> np.ndarray:
+    """Value of each e4m3 byte code, as float64 (every e4m3 value is exact).
+
+    Field by field: sign s = bit 7, exponent e = bits 6..3, mantissa m = bits
+    2..0.  e = 0: (-1)^s * m/8 * 2^-6 (subnormal); 0 < e: (-1)^s * (1 + m/8) *
+    2^(e-7); e = 15 and m = 7 is NaN (the format has no infinities, so
+    e = 15, m < 7 are ordinary values up to 448).
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = sign * val
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def attention_forward_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float, causal: bool,
+                          scale: float, row_chunk: int | None = None):
+    """Attention of e4m3-coded inputs: decode each code, multiply by the
+    tensor's descale factor, then the plain definition (attention_forward)."""
+    q = fp8_e4m3_decode(q8) * float(q_descale)
+    k = fp8_e4m3_decode(k8) * float(k_descale)
+    v = fp8_e4m3_decode(v8) * float(v_descale)
+    return attention_forward(q, k, v, causal, scale, row_chunk=row_chunk)

@@ -419,6 +419,57 @@ def pin_chunked_equals_whole(o):
     assert np.max(np.abs(whole_o[L - 1] - dec_o[0])) < 1e-12 and np.max(np.abs(whole_l[L - 1] - dec_l[0])) < 1e-12
 
 
+# -- FP8 (e4m3) inputs ---------------------------------------------------------
+
+def pin_fp8_code_points(o):
+    """e4m3 code points worked out by hand from the format's fields."""
+    with open(os.path.join(GOLDEN, "fp8_e4m3_codes.json")) as f:
+        ex = json.load(f)
+    codes = np.array([int(c["code"], 16) for c in ex["codes"]], dtype=np.uint8)
+    got = o.fp8_e4m3_decode(codes)
+    for c, g in zip(ex["codes"], got):
+        if c["value"] == "nan":
+            assert np.isnan(g)
+        else:
+            assert g == c["value"] and math.copysign(1.0, g) == math.copysign(1.0, c["value"]), (c, g)
+
+
+def pin_fp8_matches_library(o):
+    """All 256 codes against PyTorch's float8_e4m3fn conversion (a library
+    special case of the same format)."""
+    c = np.arange(256, dtype=np.uint8)
+    got = o.fp8_e4m3_decode(c)
+    ref = torch.from_numpy(c).view(torch.float8_e4m3fn).double().numpy()
+    assert np.all((got == ref) | (np.isnan(got) & np.isnan(ref)))
+
+
+def pin_fp8_attention(o):
+    """FP8 attention: scalar brute force over the decoded codes on a tiny
+    case; descales of Q and K act as a factor on the scores, the V descale
+    scales O and leaves LSE alone."""
+    rng = _rng(33)
+
+    def codes(*shape):  # sign, exponent field 0..8 (|value| < 4), any mantissa
+        return (rng.integers(0, 2, shape) * 128 + rng.integers(0, 9, shape) * 8 +
+                rng.integers(0, 8, shape)).astype(np.uint8)
+    q8, k8, v8 = codes(1, 2, 6, 4), codes(1, 1, 6, 4), codes(1, 1, 6, 4)
+    out, lse = o.attention_forward_fp8(q8, k8, v8, 0.5, 0.25, 2.0, True, 0.3)
+    dq = torch.from_numpy(q8).view(torch.float8_e4m3fn).double().numpy() * 0.5
+    dk = torch.from_numpy(k8).view(torch.float8_e4m3fn).double().numpy() * 0.25
+    dv = torch.from_numpy(v8).view(torch.float8_e4m3fn).double().numpy() * 2.0
+    for h in range(2):
+        for i in range(6):
+            w = [math.exp(0.3 * math.fsum(dq[0, h, i, c] * dk[0, 0, j, c] for c in range(4))) for j in range(i + 1)]
+            z = math.fsum(w)
+            for c in range(4):
+                want = math.fsum(wj * dv[0, 0, j, c] for j, wj in enumerate(w)) / z
+                assert abs(out[0, h, i, c] - want) <= 1e-12 * max(1.0, abs(want))
+            assert abs(lse[0, h, i] - math.log(z)) < 1e-12
+    o2, l2 = o.attention_forward_fp8(q8, k8, v8, 1.0, 1.0, 1.0, True, 0.3 * 0.5 * 0.25)
+    assert np.max(np.abs(out - 2.0 * o2)) <= 1e-12 * max(1.0, np.max(np.abs(out)))
+    assert np.max(np.abs(lse - l2)) < 1e-12
+
+
 ALL_PINS = [
     pin_rows_sum_to_one,
     pin_constant_v,
@@ -436,4 +487,7 @@ ALL_PINS = [
     pin_paged_prefill_sdpa,
     pin_paged_prefill_brute,
     pin_chunked_equals_whole,
+    pin_fp8_code_points,
+    pin_fp8_matches_library,
+    pin_fp8_attention,
 ]

@@ -233,6 +233,29 @@ def _mut_prefill_queries_from_start(m):
     m.paged_prefill = f
 
 
+def _mut_fp8_bias8(m):
+    orig = m.fp8_e4m3_decode
+    m.fp8_e4m3_decode = lambda c: orig(c) / 2.0
+
+
+def _mut_fp8_no_subnormals(m):
+    orig = m.fp8_e4m3_decode
+    def f(c):
+        c = np.asarray(c, dtype=np.uint8)
+        v = orig(c)
+        e = (c.astype(np.int64) >> 3) & 0xF
+        mm = c.astype(np.int64) & 7
+        sign = np.where(c & 0x80, -1.0, 1.0)
+        return np.where(e == 0, sign * (1 + mm / 8.0) * 2.0 ** -7, v)
+    m.fp8_e4m3_decode = f
+
+
+def _mut_fp8_v_descale_ignored(m):
+    orig = m.attention_forward_fp8
+    m.attention_forward_fp8 = lambda q8, k8, v8, qd, kd, vd, causal, scale, row_chunk=None: orig(
+        q8, k8, v8, qd, kd, 1.0, causal, scale, row_chunk)
+
+
 MUTANTS = [
     _mut_drop_scale,
     _mut_scale_squared,
@@ -252,6 +275,9 @@ MUTANTS = [
     _mut_append_ignores_table,
     _mut_prefill_no_offset,
     _mut_prefill_queries_from_start,
+    _mut_fp8_bias8,
+    _mut_fp8_no_subnormals,
+    _mut_fp8_v_descale_ignored,
 ]
 
 
