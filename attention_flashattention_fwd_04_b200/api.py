@@ -53,6 +53,8 @@ SIGNATURES = {
     "paged_attn_decode_graph_launch": (_c_i, [_c_p, _c_p]),
     "paged_attn_decode_graph_destroy": (_c_i, [_c_p]),
     "attn_device_status": (_c_i, [_c_p, ctypes.POINTER(ctypes.c_uint)]),
+    "attn_fwd_fp8": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_f, _c_f, _c_f,
+                            _c_p]),
     "paged_kv_append": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
                                _c_i, _c_p]),
     "paged_prefill": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
@@ -398,4 +400,36 @@ def paged_prefill_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tens
                                     page_size, max_pages, num_pages, int(bool(causal)), float(scale),
                                     _stream_handle(stream))
     _check(rc, "paged_prefill_append")
+    return out, lse
+
+
+def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, scale: float | None = None,
+                 q_descale: float = 1.0, k_descale: float = 1.0, v_descale: float = 1.0,
+                 out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
+    """Fused attention forward with e4m3 inputs: q [B,Hq,N,128], k/v
+    [B,Hkv,N,128] as torch.float8_e4m3fn (or their uint8 codes); the
+    attention is over q*q_descale, k*k_descale, v*v_descale.
+    Returns (o [B,Hq,N,128] bf16, lse [B,Hq,N] fp32)."""
+    def codes(t, name):
+        if isinstance(t, torch.Tensor) and t.dtype == torch.float8_e4m3fn:
+            t = t.view(torch.uint8)
+        _require(t, name, torch.uint8, 4)
+        return t
+    q, k, v = codes(q, "q"), codes(k, "k"), codes(v, "v")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} do not match q {tuple(q.shape)}")
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    if out is None:
+        out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _require(out, "out", torch.bfloat16, 4)
+    _require(lse, "lse", torch.float32, 3)
+    rc = lib().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N,
+                            d, int(bool(causal)), float(scale), float(q_descale), float(k_descale), float(v_descale),
+                            _stream_handle(stream))
+    _check(rc, "attn_fwd_fp8")
     return out, lse

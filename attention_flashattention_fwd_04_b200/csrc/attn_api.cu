@@ -48,14 +48,15 @@ EncodeTiledFn encode_fn() {
 // dims[0] is the contiguous dimension; strides are the byte strides of
 // dims[1] and dims[2].
 bool encode_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
-               uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2) {
+               uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2,
+               CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
   const cuuint64_t strides[2] = {stride1, stride2};
   const cuuint32_t box[3] = {b0, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+  const CUresult r = fn(map, dtype, 3, const_cast<void*>(ptr), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -93,12 +94,12 @@ int sm_count() {
   return counts[dev];
 }
 
-template <int D, bool CAUSAL, bool WINDOW, bool PAGED = false>
+template <int D, bool CAUSAL, bool WINDOW, bool PAGED = false, bool FP8 = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const attn::PrefillParams& p, cudaStream_t stream) {
-  using L = attn::PrefillLayout<D, PAGED>;
-  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED>;
-  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED>>(L::kAlloc);
+  using L = attn::PrefillLayout<D, PAGED, FP8>;
+  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED, FP8>;
+  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED, FP8>>(L::kAlloc);
   if (e != cudaSuccess) return fail_cuda(e);
   const int sms = sm_count();
   if (sms <= 0) return fail_cuda(cudaErrorInvalidDevice);
@@ -251,6 +252,7 @@ int attn_fwd_window(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, 
   p.num_items = static_cast<int>(blocks * bh);
   p.window_left = window_left >= N - 1 ? -1 : window_left;  // a window covering every key is no window
   p.scale_log2 = scale * kLog2e;
+  p.o_scale = 1.f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool win = p.window_left >= 0;
   if (d == 128) {
@@ -576,6 +578,7 @@ int launch_paged_prefill(const attn_bf16* q, const attn_bf16* k_pool, const attn
   p.num_items = 0;
   p.window_left = -1;
   p.scale_log2 = scale * kLog2e;
+  p.o_scale = 1.f;
   p.cu_q = cu_seqlens_q;
   p.seq_lens = seq_lens;
   p.block_table = block_table;
@@ -641,3 +644,60 @@ int paged_prefill_append(const attn_bf16* q, const attn_bf16* k_new, const attn_
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// FP8 (e4m3) prefill
+// ----------------------------------------------------------------------------
+
+extern "C" {
+
+int attn_fwd_fp8(const uint8_t* q, const uint8_t* k, const uint8_t* v, attn_bf16* o, float* lse, int B, int Hq,
+                 int Hkv, int N, int d, int causal, float scale, float q_descale, float k_descale, float v_descale,
+                 void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_SHAPE;
+  if (d != 64 && d != 128) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return ATTN_ERR_SHAPE;
+  for (const float x : {scale, q_descale, k_descale, v_descale})
+    if (!(x > 0.f) || !std::isfinite(x)) return ATTN_ERR_SHAPE;
+  if (!std::isfinite(scale * q_descale * k_descale * kLog2e)) return ATTN_ERR_SHAPE;
+  const long long bh = static_cast<long long>(B) * Hq;
+  const long long blocks = (static_cast<long long>(N) + 255) / 256;
+  if (bh > INT_MAX || blocks * bh > INT_MAX) return ATTN_ERR_SHAPE;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;  // an e4m3 row of 128 is exactly one 128-byte swizzled box
+  if (misaligned16(q) || misaligned16(k) || misaligned16(v) || misaligned16(o) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
+    return ATTN_ERR_ALIGN;
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t row_bytes = static_cast<uint64_t>(d);  // one byte per element
+  const uint64_t head_bytes = row_bytes * static_cast<uint64_t>(N);
+  if (!encode_3d(&tq, q, d, N, static_cast<uint64_t>(B) * Hq, row_bytes, head_bytes, 128, 128, 1,
+                 CU_TENSOR_MAP_DATA_TYPE_UINT8) ||
+      !encode_3d(&tk, k, d, N, static_cast<uint64_t>(B) * Hkv, row_bytes, head_bytes, 128, 128, 1,
+                 CU_TENSOR_MAP_DATA_TYPE_UINT8) ||
+      !encode_3d(&tv, v, d, N, static_cast<uint64_t>(B) * Hkv, row_bytes, head_bytes, 128, 128, 1,
+                 CU_TENSOR_MAP_DATA_TYPE_UINT8))
+    return fail_cuda(cudaErrorInvalidValue);
+
+  attn::PrefillParams p{};
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.num_m = static_cast<int>(blocks);
+  p.num_items = static_cast<int>(blocks * bh);
+  p.window_left = -1;
+  p.scale_log2 = scale * q_descale * k_descale * kLog2e;
+  p.o_scale = v_descale;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return causal ? launch_prefill<128, true, false, false, true>(tq, tk, tv, p, s)
+                : launch_prefill<128, false, false, false, true>(tq, tk, tv, p, s);
+}
+
+}  // extern "C"
+

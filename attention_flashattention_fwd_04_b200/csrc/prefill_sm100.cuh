@@ -67,7 +67,8 @@ struct PrefillParams {
   int num_m;         // ceil(N / 256): 256-row query blocks per head
   int num_items;     // B * Hq * num_m (paged: counted on the device)
   int window_left;   // query i sees keys >= i - window_left (kernels with WINDOW only)
-  float scale_log2;  // scale * log2(e)
+  float scale_log2;  // scale * log2(e) (FP8: times the Q and K descales)
+  float o_scale;     // FP8: the V descale, applied to O in the epilogue
   // Paged prefill (kernels with PAGED only): the new queries of sequence s
   // are packed rows cu_q[s] .. cu_q[s+1]-1; the cache holds seq_lens[s]
   // tokens of it (the new ones last), read through block_table.
@@ -85,13 +86,22 @@ constexpr int kPagedMaxBlocks = 2048;  // 256-row query blocks per paged-prefill
 
 constexpr int kPrefillThreads = 512;
 constexpr float kRescaleThreshold = 8.0f;  // in log2 units
+// FP8: P is stored as e4m3 scaled by 2^8 (so that the weights of keys a few
+// units below the row max stay normal numbers), and the stale max may lag the
+// true one by at most 0.5, so 2^8 * 2^0.5 = 362 stays below e4m3's 448.
+constexpr float kFp8PLog2 = 8.0f;
+constexpr float kRescaleThresholdFp8 = 0.5f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D, bool PAGED = false>
+template <int D, bool PAGED = false, bool FP8 = false>
 struct PrefillLayout {
-  static constexpr int NS = 2;                 // K and V ring depth
-  static constexpr int kBoxBytes = 128 * 128;  // 128 rows x 64 bf16 (one 128B-swizzled box)
-  static constexpr int kTileBytes = 128 * D * 2;
+  static_assert(!FP8 || D == 128, "FP8 tiles are one 128-byte box wide");
+  static constexpr int NS = 2;                     // K and V ring depth
+  static constexpr int kElemBytes = FP8 ? 1 : 2;   // bf16 or e4m3
+  static constexpr int kBoxCols = 128 / kElemBytes;  // elements per 128-byte swizzled row
+  static constexpr int kBoxes = D / kBoxCols;        // boxes across the head dim
+  static constexpr int kBoxBytes = 128 * 128;      // 128 rows x 128 bytes (one 128B-swizzled box)
+  static constexpr int kTileBytes = 128 * D * kElemBytes;
   static constexpr int kQ0 = 0;
   static constexpr int kQ1 = kTileBytes;
   static constexpr int kK = 2 * kTileBytes;
@@ -351,14 +361,15 @@ __device__ __forceinline__ void reg_alloc_control() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
 }
 
-template <int D, bool CAUSAL, bool WINDOW, bool PAGED>
+template <int D, bool CAUSAL, bool WINDOW, bool PAGED, bool FP8 = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(!(PAGED && WINDOW), "the paged kernels have no window");
-  using L = PrefillLayout<D, PAGED>;
+  static_assert(!(FP8 && (PAGED || WINDOW)), "the FP8 kernels are dense, without a window");
+  using L = PrefillLayout<D, PAGED, FP8>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -443,8 +454,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if constexpr (!PAGED) {
           if (lane == 0) {
             mbar_arrive_expect_tx(full, L::kTileBytes);
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(dst + c * L::kBoxBytes, map, full, c * 64, j * 128, kz);
+            for (int c = 0; c < L::kBoxes; ++c)
+              tma_load_3d(dst + c * L::kBoxBytes, map, full, c * L::kBoxCols, j * 128, kz);
           }
         } else {
           // Box b (lane b) holds keys 128j + b*pb ...: a page (or a 128-key
@@ -556,11 +567,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (r > 0 && !(ok = wait0(bar(L::kBarQEmpty), static_cast<uint32_t>(r - 1) & 1u, kErrWaitQ))) break;
         if (lane == 0) {
           mbar_arrive_expect_tx(bar(L::kBarQFull), (it.has(1) ? 2 : 1) * L::kTileBytes);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(base + L::kQ0 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, qrow, qz);
+          for (int c = 0; c < L::kBoxes; ++c)
+            tma_load_3d(base + L::kQ0 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * L::kBoxCols, qrow, qz);
           if (it.has(1))
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(base + L::kQ1 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * 64, qrow + 128, qz);
+            for (int c = 0; c < L::kBoxes; ++c)
+              tma_load_3d(base + L::kQ1 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * L::kBoxCols, qrow + 128,
+                          qz);
         }
         ++q_issued;
         if (!(ok = load_v(it.jb, kz))) break;
@@ -582,8 +594,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       __syncwarp();
     } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idesc_pv = make_idesc_bf16(128, D, false, true);
+      constexpr uint32_t idesc_qk =
+          FP8 ? make_idesc_e4m3(128, 128, false, false) : make_idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_pv = FP8 ? make_idesc_e4m3(128, D, false, true) : make_idesc_bf16(128, D, false, true);
+      // Every MMA takes 32 bytes of its K dimension: 16 bf16 or 32 e4m3.
+      constexpr int kSSteps = D * L::kElemBytes / 32;     // S = Q K^T over the head dim
+      constexpr int kPvKeys = 32 / L::kElemBytes;         // keys per P V step
+      constexpr int kPvSteps = 128 / kPvKeys;
       int kv_it = 0;
       uint32_t p_cnt[2] = {0u, 0u};
       uint32_t o_cnt[2] = {0u, 0u};  // items whose O_t has been completed
@@ -593,10 +610,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t k_addr = base + L::kK + st * L::kTileBytes;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(t) * 128u;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < kSSteps; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk >> 2) * L::kBoxBytes + (kk & 3) * 32);
-          mma_bf16_ss(d_tmem, make_sdesc_sw128(q_addr + off, 16, 1024),
-                      make_sdesc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          if constexpr (FP8)
+            mma_f8_ss(d_tmem, make_sdesc_sw128(q_addr + off, 16, 1024), make_sdesc_sw128(k_addr + off, 16, 1024),
+                      idesc_qk, kk > 0 ? 1u : 0u);
+          else
+            mma_bf16_ss(d_tmem, make_sdesc_sw128(q_addr + off, 16, 1024),
+                        make_sdesc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(L::kBarSFull + t));
       };
@@ -605,9 +626,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t p_tmem = tmem + static_cast<uint32_t>(t) * 128u;
         const uint32_t o_tmem = tmem + L::kColO + static_cast<uint32_t>(t * D);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(o_tmem, p_tmem + kk * 8, make_sdesc_sw128(v_addr + kk * 2048, L::kBoxBytes, 1024),
-                      idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kPvSteps; ++kk) {
+          // P: 32 bytes of a row per step = 8 TMEM columns; V: kPvKeys rows of 128 bytes.
+          const uint64_t vdesc = make_sdesc_sw128(v_addr + kk * kPvKeys * 128, L::kBoxBytes, 1024);
+          if constexpr (FP8)
+            mma_f8_ts(o_tmem, p_tmem + kk * 8, vdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+          else
+            mma_bf16_ts(o_tmem, p_tmem + kk * 8, vdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+        }
       };
       PrefillItem it;
       for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
@@ -707,7 +733,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_arrive(bar(L::kBarStatsEmpty + 2 * t + slot));
         ++st_cnt[t];
         const int grow = it.m * 256 + t * 128 + row;  // query row of the head (paged: of the sequence's chunk)
-        const float inv_l = 1.f / l_sum;
+        const float inv_l = (FP8 ? p.o_scale : 1.f) / l_sum;  // FP8: l carries P's 2^8 as O does
         // O row / LSE index: dense [B, Hq, N, D] / [B, Hq, N]; paged by token, [total_q, Hq, D] / [total_q, Hq].
         const bool valid = grow < (PAGED ? it.n_q : p.N);
         const size_t row_index = PAGED ? (static_cast<size_t>(it.q0) + grow) * p.Hq + it.h
@@ -729,7 +755,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
           }
         }
-        if (valid) p.lse[row_index] = (m_used + log2f(l_sum)) * kLn2;
+        if (valid) p.lse[row_index] = (m_used + log2f(l_sum) - (FP8 ? kFp8PLog2 : 0.f)) * kLn2;
         tc_fence_before();
         mbar_arrive(bar(L::kBarOFree + t));
       }
@@ -785,23 +811,29 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               if (c > last) s[c] = -INFINITY;
           }
         }
-        // Row max: four chains of three-input maxima.
+        // Row max: four chains of three-input maxima over s[4..123], then
+        // s[124..127] one per chain.
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 128; c += 8) {
+        for (int c = 4; c + 8 <= 124; c += 8) {
           mx0 = max3(mx0, s[c], s[c + 1]);
           mx1 = max3(mx1, s[c + 2], s[c + 3]);
           mx2 = max3(mx2, s[c + 4], s[c + 5]);
           mx3 = max3(mx3, s[c + 6], s[c + 7]);
         }
+        mx0 = fmaxf(mx0, s[124]);
+        mx1 = fmaxf(mx1, s[125]);
+        mx2 = fmaxf(mx2, s[126]);
+        mx3 = fmaxf(mx3, s[127]);
         float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
         m_tile *= sl2;
         const float m_new = fmaxf(m_used, m_tile);
-        const bool upd = m_new > m_used + kRescaleThreshold;
+        const bool upd = m_new > m_used + (FP8 ? kRescaleThresholdFp8 : kRescaleThreshold);
         const float alpha = upd ? ex2_approx(m_used - m_new) : 1.f;  // 0 on the first tile
         if (upd) m_used = m_new;
         l_sum *= alpha;
-        const float neg_m = (m_used == -INFINITY) ? 0.f : -m_used;
+        // FP8: P = 2^8 * 2^(s - m), the 2^8 folded into the offset.
+        const float neg_m = (m_used == -INFINITY) ? 0.f : (FP8 ? kFp8PLog2 - m_used : -m_used);
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
         const uint64_t negm2 = f2_pack(neg_m, neg_m);
         // P in two halves, columns [0, 64) then [64, 128); each half goes to
@@ -809,24 +841,42 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+          if constexpr (FP8) {
+            // Four e4m3 weights per 32-bit column: 16 columns per half.
+            uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int c = half * 64 + 2 * i;
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2), x0, x1);
-            float p0, p1;
-            if (kExp2EmuPeriod > 0 && i % (kExp2EmuPeriod > 0 ? kExp2EmuPeriod : 1) == kExp2EmuPeriod - 1) {
-              p0 = exp2_poly(x0);
-              p1 = exp2_poly(x1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
+            for (int i = 0; i < 16; ++i) {
+              const int c = half * 64 + 4 * i;
+              float x0, x1, x2, x3;
+              f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2), x0, x1);
+              f2_unpack(f2_fma(f2_pack(s[c + 2], s[c + 3]), sl2x2, negm2), x2, x3);
+              const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
+              const float p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+              acc[0] = f2_add(acc[0], f2_pack(p0, p1));
+              acc[1] = f2_add(acc[1], f2_pack(p2, p3));
+              pk[i] = pack_e4m3x4(p0, p1, p2, p3);
             }
-            acc[i & 1] = f2_add(acc[i & 1], f2_pack(p0, p1));
-            pk[i] = pack_bf16x2(p0, p1);
+            tmem_st_x16(s_addr + static_cast<uint32_t>(half * 16), pk);
+          } else {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int c = half * 64 + 2 * i;
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2), x0, x1);
+              float p0, p1;
+              if (kExp2EmuPeriod > 0 && i % (kExp2EmuPeriod > 0 ? kExp2EmuPeriod : 1) == kExp2EmuPeriod - 1) {
+                p0 = exp2_poly(x0);
+                p1 = exp2_poly(x1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              acc[i & 1] = f2_add(acc[i & 1], f2_pack(p0, p1));
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st_x32(s_addr + static_cast<uint32_t>(half * 32), pk);
           }
-          tmem_st_x32(s_addr + static_cast<uint32_t>(half * 32), pk);
           if (half == 0 && jj > 0 && __any_sync(0xffffffffu, upd)) {
             // O_t is idle here (its last update was issued before S_t of this
             // tile, and this tile's update waits for the barrier below).

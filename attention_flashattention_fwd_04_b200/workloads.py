@@ -43,6 +43,7 @@ __all__ = [
     "PREFILL_CONFIGS",
     "DECODE_CONFIGS",
     "make_prefill_inputs",
+    "make_prefill_inputs_fp8",
     "make_decode_inputs",
     "ChunkedConfig",
     "CHUNKED_CONFIGS",
@@ -240,6 +241,20 @@ def make_prefill_inputs(cfg: PrefillConfig, device: str | torch.device = "cpu"):
         k.add_(off.view(1, 1, cfg.N, 1))
     out = tuple(t.to(torch.bfloat16).contiguous().to(device) for t in (q, k, v))
     return out
+
+
+def make_prefill_inputs_fp8(cfg: PrefillConfig, device: str | torch.device = "cpu"):
+    """The bf16 draw of ``cfg`` quantised to e4m3 per tensor: descale =
+    amax / 448, codes = round-to-nearest-even(x / descale) (PyTorch's
+    float8_e4m3fn conversion).  Returns (q8, k8, v8) as uint8 codes and
+    (q_descale, k_descale, v_descale) as Python floats (fp32 values)."""
+    codes, scales = [], []
+    for t in make_prefill_inputs(cfg):
+        x = t.float()
+        d = float(torch.tensor(max(float(x.abs().max()), 1e-30) / 448.0, dtype=torch.float32))
+        codes.append((x / d).to(torch.float8_e4m3fn).view(torch.uint8).contiguous().to(device))
+        scales.append(d)
+    return tuple(codes), tuple(scales)
 
 
 def make_decode_inputs(cfg: DecodeConfig, device: str | torch.device = "cpu",

@@ -100,6 +100,20 @@ int attn_fwd_window(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, 
                     float scale, void* stream);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd with e4m3 inputs (OCP FP8 E4M3 codes, one byte
+ * each, same [B, H, N, d] layouts): the attention of q * q_descale,
+ * k * k_descale and v * v_descale, the FP8 tensor-core path of FlashAttention
+ * v3 (the anylearn.cc lesson's FA v3 section).  Q K^T and P V run on the FP8
+ * tensor cores with fp32 accumulation; P is rounded to e4m3 (scaled by 2^8)
+ * before P V, the row sums and LSE use P unrounded.  o is bf16, lse fp32.
+ * d must be 128 (ATTN_ERR_UNSUPPORTED for 64); the descales finite and > 0.
+ * Error behaviour as attn_fwd.
+ */
+int attn_fwd_fp8(const uint8_t* q, const uint8_t* k, const uint8_t* v, attn_bf16* o, float* lse, int B, int Hq,
+                 int Hkv, int N, int d, int causal, float scale, float q_descale, float k_descale, float v_descale,
+                 void* stream);
+
+/*
  * paged_attn_decode_split_tokens -- tokens per split of the split-KV decode
  * pass for this problem shape (a multiple of 16).  The split plan depends only
  * on these arguments, never on the sequence lengths, so the host never has to

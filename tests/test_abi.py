@@ -171,3 +171,20 @@ def test_paged_prefill_rejects(lib, fn, kw, code):
 
 def test_paged_prefill_with_no_new_tokens_is_a_no_op(lib):
     assert _pp(lib, total_q=0) == 0
+
+
+def _fp8(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=16, d=128, causal=1, scale=0.1,
+         qd=1.0, kd=1.0, vd=1.0):
+    return lib.attn_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, qd, kd, vd, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(v=None), 1), (dict(lse=None), 1),
+    (dict(B=0), 2), (dict(N=0), 2), (dict(d=96), 2), (dict(Hq=6, Hkv=4), 2), (dict(causal=3), 2),
+    (dict(scale=0.0), 2), (dict(qd=0.0), 2), (dict(kd=-1.0), 2), (dict(vd=float("inf")), 2),
+    (dict(qd=1e30, kd=1e30), 2),
+    (dict(d=64), 5),
+    (dict(q=FAKE + 8), 3), (dict(o=FAKE + 2), 3),
+])
+def test_attn_fwd_fp8_rejects(lib, kw, code):
+    assert _fp8(lib, **kw) == code
