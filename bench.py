@@ -173,6 +173,7 @@ class ClockSampler:
 PREFILL_WORKLOADS = ("default", "causal_mha", "causal_gqa", "long_causal", "long_window", "tiny")
 DECODE_WORKLOADS = ("default", "paged_decode", "small_decode")
 CHUNKED_WORKLOADS = ("chunked_prefill",)
+FP8_WORKLOADS = {"causal_gqa_fp8": "causal_gqa", "long_causal_fp8": "long_causal"}  # e4m3 inputs, same shapes
 
 
 def chunked_label(c) -> str:
@@ -180,8 +181,8 @@ def chunked_label(c) -> str:
             f"context {c.ctx_range[0]}..{c.ctx_range[1]} new {c.q_range[0]}..{c.q_range[1]}")
 
 
-def prefill_label(c) -> str:
-    mask = "causal" if c.causal else "full"
+def prefill_label(c, fp8=False) -> str:
+    mask = ("fp8 " if fp8 else "") + ("causal" if c.causal else "full")
     if c.window_left >= 0:
         mask += f" window={c.window_left}"
     return f"{mask} prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}"
@@ -200,8 +201,9 @@ class Step:
         if workload in CHUNKED_WORKLOADS:
             base = W.CHUNKED_CONFIGS[workload]
             self.chunked_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
-        if workload in PREFILL_WORKLOADS:
-            name = "causal_mha" if workload == "default" else workload
+        self.fp8 = workload in FP8_WORKLOADS
+        if workload in PREFILL_WORKLOADS or self.fp8:
+            name = "causal_mha" if workload == "default" else FP8_WORKLOADS.get(workload, workload)
             base = W.PREFILL_CONFIGS[name]
             self.prefill_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
         if workload in DECODE_WORKLOADS:
@@ -214,7 +216,10 @@ class Step:
         self.bytes = 0.0
         if self.prefill_cfg is not None:
             c = self.prefill_cfg
-            q, k, v = W.make_prefill_inputs(c)
+            if self.fp8:
+                (q, k, v), self.descales = W.make_prefill_inputs_fp8(c)
+            else:
+                q, k, v = W.make_prefill_inputs(c)
             self.host.update(q=q, k=k, v=v)
             self.flops = W.prefill_flops(c)
         if self.decode_cfg is not None:
@@ -249,7 +254,7 @@ class Step:
         api, dev = self.api, self.device
         if self.prefill_cfg is not None:
             q = self.dev["q"]
-            self.dev["o"] = torch.empty_like(q)
+            self.dev["o"] = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
             self.dev["lse"] = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
         if self.chunked_cfg is not None:
             q = self.dev["cq"]
@@ -289,6 +294,10 @@ class Step:
     def run_prefill(self, d=None):
         d = d or self.dev
         c = self.prefill_cfg
+        if self.fp8:
+            qd, kd, vd = self.descales
+            self.api.attn_fwd_fp8(d["q"], d["k"], d["v"], c.causal, c.scale, qd, kd, vd, out=d["o"], lse=d["lse"])
+            return
         self.api.attn_fwd(d["q"], d["k"], d["v"], c.causal, c.scale, out=d["o"], lse=d["lse"],
                           window_left=c.window_left if c.window_left >= 0 else None)
 
@@ -301,8 +310,14 @@ class Step:
         self.api.paged_attn_decode(d["dq"], d["k_pool"], d["v_pool"], d["block_table"], d["seq_lens"], c.scale,
                                    workspace=self.dev["ws"], out=d["do"], lse=d["dlse"])
 
+    def tensor_peak_tflops(self, peaks) -> float:
+        """Peak for this step's contraction dtype: the measured bf16 GEMM
+        rate, doubled for e4m3 (the nominal dense fp8 / bf16 ratio, 4.5 / 2.25
+        PFLOP/s)."""
+        return peaks["bf16_tflops"] * (2.0 if self.fp8 else 1.0)
+
     def ideal_seconds(self, peaks) -> float:
-        return self.flops / (peaks["bf16_tflops"] * 1e12) + self.bytes / (peaks["hbm_gbs"] * 1e9)
+        return self.flops / (self.tensor_peak_tflops(peaks) * 1e12) + self.bytes / (peaks["hbm_gbs"] * 1e9)
 
 
 def config_dict(step: Step, n_gpus: int):
@@ -310,10 +325,11 @@ def config_dict(step: Step, n_gpus: int):
     parts = []
     if step.prefill_cfg is not None:
         c = step.prefill_cfg
-        parts.append(prefill_label(c))
+        parts.append(prefill_label(c, step.fp8))
         cfg["prefill"] = {"B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "N": c.N, "d": c.d, "causal": c.causal,
                           "window_left": c.window_left, "scale": c.scale, "seed": c.seed,
-                          "value_scale": c.value_scale, "k_offset_sigma": c.k_offset_sigma, "flops": step.flops}
+                          "value_scale": c.value_scale, "k_offset_sigma": c.k_offset_sigma, "flops": step.flops,
+                          "inputs": "e4m3, per-tensor descale amax/448" if step.fp8 else "bf16"}
     if step.chunked_cfg is not None:
         c, inp = step.chunked_cfg, step.chunked_inp
         parts.append(chunked_label(c))
@@ -352,7 +368,7 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
 
     import oracle
 
-    prefill_cfg, decode_cfg, host, decode_inp, chunked = step_cfgs
+    prefill_cfg, decode_cfg, host, decode_inp, chunked, fp8 = step_cfgs
     flops = 0.0
     nbytes = 0.0
     done_heads = 0
@@ -385,7 +401,10 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
                 break
     if prefill_cfg is not None:
         c = prefill_cfg
-        q, k, v = (host[n].float().numpy() for n in ("q", "k", "v"))
+        if fp8 is not None:  # e4m3 codes: the oracle decodes them (timed: it is the oracle's work)
+            q, k, v = (oracle.fp8_e4m3_decode(host[n].numpy()) * dsc for n, dsc in zip(("q", "k", "v"), fp8))
+        else:
+            q, k, v = (host[n].float().numpy() for n in ("q", "k", "v"))
         rows = c.N if not per_call else 128
         for b in range(c.B):
             for h in range(c.Hq):
@@ -450,7 +469,7 @@ def run_reference(args, world, rank):
         return None
     peaks = load_peaks()
     step = StepHost(args.workload)
-    cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp, step.chunked)
+    cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp, step.chunked, step.fp8)
     for _ in range(args.warmup):
         oracle_sample(cfgs, 0.0, per_call=True)
     work_f = work_b = secs = 0.0
@@ -460,7 +479,8 @@ def run_reference(args, world, rank):
         work_f += w["flops"]
         work_b += w["bytes"]
         secs += s
-    ideal = work_f / (peaks["bf16_tflops"] * 1e12) + work_b / (peaks["hbm_gbs"] * 1e9)
+    tpk = peaks["bf16_tflops"] * (2.0 if step.fp8 is not None else 1.0)  # e4m3: nominal 2x bf16
+    ideal = work_f / (tpk * 1e12) + work_b / (peaks["hbm_gbs"] * 1e9)
     value = ideal / secs
     line = {
         "metric": METRIC, "value": value, "unit": unit_string(), "n_gpus": world, "steps": args.steps,
@@ -482,7 +502,13 @@ class StepHost:
         self.host = {}
         self.decode_inp = None
         self.chunked = None
+        self.fp8 = None
         parts = []
+        if workload in FP8_WORKLOADS:
+            self.prefill_cfg = W.PREFILL_CONFIGS[FP8_WORKLOADS[workload]]
+            (q, k, v), self.fp8 = W.make_prefill_inputs_fp8(self.prefill_cfg)
+            self.host.update(q=q, k=k, v=v)
+            parts.append(prefill_label(self.prefill_cfg, True))
         if workload in CHUNKED_WORKLOADS:
             c = W.CHUNKED_CONFIGS[workload]
             self.chunked = (c, W.make_chunked_inputs(c))
@@ -505,7 +531,8 @@ class StepHost:
 
 
 def unit_string() -> str:
-    return "fraction of B200 peak (time-weighted: prefill bf16 FLOP/s, decode HBM B/s), summed over GPUs"
+    return ("fraction of B200 peak (time-weighted: prefill tensor FLOP/s at the inputs' dtype peak, "
+            "decode/append HBM B/s), summed over GPUs")
 
 
 def run_ours(args, world, rank, local_rank):
@@ -590,7 +617,7 @@ def run_ours(args, world, rank, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": unit_string(), "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t_max / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if step.fp8 else "bf16", "data": "synthetic",
         "config": config_dict(step, world),
         "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clocks.summary(),
@@ -600,8 +627,9 @@ def run_ours(args, world, rank, local_rank):
     if step.prefill_cfg is not None:
         per = t_prefill / args.steps
         tfl = step.flops / per / 1e12
-        kernels["prefill_fwd_kernel"] = {"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"],
-                                         "unit": "TFLOP/s", "frac": tfl / peaks["bf16_tflops"],
+        tpk = step.tensor_peak_tflops(peaks)
+        kernels["prefill_fwd_kernel"] = {"bound": "tensor", "achieved": tfl, "peak": tpk,
+                                         "unit": "TFLOP/s", "frac": tfl / tpk,
                                          "us_per_launch": per * 1e6, "algorithmic": step.flops}
         line["prefill_tflops"] = tfl
     if step.decode_cfg is not None:
@@ -635,16 +663,19 @@ def run_ours(args, world, rank, local_rank):
     else:
         parts = [traffic.get((k, step.decode_cfg.name)) for k in ("decode_split_kernel", "decode_merge_kernel")]
         tr = None if any(x is None for x in parts) else sum(parts)
+    peak_source = f"{peaks['source']} (burst)"
+    if step.fp8 and dominant.startswith("prefill"):
+        peak_source += ", bf16 x 2 (nominal e4m3 / bf16 dense ratio)"
     line["roofline"] = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
-                        "unit": dk["unit"], "frac": dk["frac"], "traffic": tr,
-                        "peak_source": f"{peaks['source']} (burst)"}
+                        "unit": dk["unit"], "frac": dk["frac"], "traffic": tr, "peak_source": peak_source}
     line["kernels"] = kernels
     line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         chunked = (step.chunked_cfg, step.chunked_inp) if step.chunked_cfg is not None else None
         w, secs, desc = oracle_sample((step.prefill_cfg, step.decode_cfg, step.host,
-                                       getattr(step, "decode_inp", None), chunked), args.cpu_seconds)
-        ideal = w["flops"] / (peaks["bf16_tflops"] * 1e12) + w["bytes"] / (peaks["hbm_gbs"] * 1e9)
+                                       getattr(step, "decode_inp", None), chunked,
+                                       step.descales if step.fp8 else None), args.cpu_seconds)
+        ideal = w["flops"] / (step.tensor_peak_tflops(peaks) * 1e12) + w["bytes"] / (peaks["hbm_gbs"] * 1e9)
         cpu = {"value": ideal / secs, "unit": unit_string(), "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{desc}; {secs:.1f} s"}
         if w["flops"]:
@@ -705,7 +736,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="default",
-                    choices=sorted(set(PREFILL_WORKLOADS) | set(DECODE_WORKLOADS) | set(CHUNKED_WORKLOADS)))
+                    choices=sorted(set(PREFILL_WORKLOADS) | set(DECODE_WORKLOADS) | set(CHUNKED_WORKLOADS) |
+                                   set(FP8_WORKLOADS)))
     ap.add_argument("--decode-graph", action="store_true",
                     help="run the decode step as a captured CUDA graph (split pass + merge)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
