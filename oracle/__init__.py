@@ -10,6 +10,7 @@ from .attention import (  # noqa: F401
     attention_head,
     attention_rows,
     attention_scores,
+    block_keep,
     fp8_e4m3_decode,
     gather_paged_kv,
     gqa_kv_head,

@@ -35,6 +35,12 @@ Readings where the pages are silent (each is restated where it is used):
   t % page_size ("Paged Attention Kernels" section and its block-table figure,
   logical blocks 0,1,2,3 -> physical 17,4,29,8).  Decode has one query per
   sequence that sees all seq_len cached keys.
+* block-sparse masks (FlashInfer's 2-D block-sparse masks in "Kernel Fusion
+  and Custom Kernels", section 4, e.g. the Longformer pattern): a boolean
+  [B, Hq, ceil(N/128), ceil(N/128)] block mask; M = -inf for every key of a
+  masked 128 x 128 block, on top of the causal mask.  A row that sees no key
+  at all outputs zeros with LSE = -inf (the pages leave it open; this is the
+  decode's convention for an empty sequence).
 * FP8 inputs (the anylearn.cc lesson's FA v3 section: Q K^T and P V computed
   in FP8): Q, K, V arrive as e4m3 codes with one descale factor per tensor;
   the operation is attention over the decoded values times their descales
@@ -69,6 +75,7 @@ import numpy as np
 
 __all__ = [
     "gqa_kv_head",
+    "block_keep",
     "attention_scores",
     "softmax_with_lse",
     "attention_head",
@@ -100,7 +107,7 @@ def gqa_kv_head(h_q: int, Hq: int, Hkv: int) -> int:
 
 
 def attention_scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
-                     row_offset: int = 0, window_left: int | None = None) -> np.ndarray:
+                     row_offset: int = 0, window_left: int | None = None, keep=None) -> np.ndarray:
     """S = scale * q k^T + M for one head.
 
     ``q`` holds query rows ``row_offset .. row_offset + len(q) - 1`` of the head;
@@ -119,6 +126,8 @@ def attention_scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
         s = np.where(cols > rows, -np.inf, s)
     if window_left is not None and window_left >= 0:
         s = np.where(cols < rows - int(window_left), -np.inf, s)
+    if keep is not None:  # boolean [len(q), len(k)]: False -> -inf
+        s = np.where(np.asarray(keep, dtype=bool), s, -np.inf)
     return s
 
 
@@ -131,27 +140,41 @@ def softmax_with_lse(s: np.ndarray):
     """
     s = _f64(s)
     m = np.max(s, axis=-1, keepdims=True)
-    lse = m + np.log(np.sum(np.exp(s - m), axis=-1, keepdims=True))
-    p = np.exp(s - lse)
+    empty = np.isneginf(m)  # a row with no visible key: P = 0, LSE = -inf
+    m = np.where(empty, 0.0, m)
+    with np.errstate(divide="ignore"):  # log(0) = -inf is the intended LSE of an empty row
+        lse = m + np.log(np.sum(np.exp(s - m), axis=-1, keepdims=True))
+    p = np.where(empty, 0.0, np.exp(s - np.where(empty, 0.0, lse)))
     return p, lse[..., 0]
 
 
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
-                   causal: bool, row_offset: int = 0, window_left: int | None = None):
+                   causal: bool, row_offset: int = 0, window_left: int | None = None, keep=None):
     """O and LSE for one head: materialise S, then P, then O = P V."""
-    s = attention_scores(q, k, scale, causal, row_offset, window_left)
+    s = attention_scores(q, k, scale, causal, row_offset, window_left, keep)
     p, lse = softmax_with_lse(s)
     o = p @ _f64(v)
     return o, lse
 
 
+def block_keep(block_mask_bh, rows, n_keys: int, block: int = 128) -> np.ndarray:
+    """Element mask of query rows `rows` over keys 0..n_keys-1 from one head's
+    [q_blocks, k_blocks] block mask: key j is kept for row i iff block
+    (i // block, j // block) is set."""
+    bm = np.asarray(block_mask_bh, dtype=bool)
+    rows = np.asarray(rows, dtype=np.int64)
+    cols = np.arange(int(n_keys))
+    return bm[rows[:, None] // block, cols[None, :] // block]
+
+
 def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None = None,
-                      window_left: int | None = None):
+                      window_left: int | None = None, block_mask=None):
     """Full attention forward for [B, Hq, N, d] queries and [B, Hkv, N, d] K/V.
 
     Returns (O [B, Hq, N, d] float64, LSE [B, Hq, N] float64).  ``row_chunk``
     splits each head into blocks of complete query rows (every row still sees
     its whole key set), which only bounds memory for long sequences.
+    ``block_mask``: boolean [B, Hq, ceil(N/128), ceil(N/128)] (see block_keep).
     """
     q = _f64(q)
     k = _f64(k)
@@ -166,14 +189,15 @@ def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None
             hk = gqa_kv_head(h, Hq, Hkv)
             for r0 in range(0, N, step):
                 r1 = min(N, r0 + step)
+                keep = None if block_mask is None else block_keep(block_mask[b, h], np.arange(r0, r1), N)
                 o[b, h, r0:r1], lse[b, h, r0:r1] = attention_head(
                     q[b, h, r0:r1], k[b, hk], v[b, hk], scale, causal, row_offset=r0,
-                    window_left=window_left)
+                    window_left=window_left, keep=keep)
     return o, lse
 
 
 def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows,
-                   window_left: int | None = None):
+                   window_left: int | None = None, block_mask=None):
     """O and LSE of selected query rows of head (b, h), each row exact.
 
     Used for sampled parity checks at sizes where the full oracle is too slow.
@@ -187,7 +211,9 @@ def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows,
     out_l = np.empty(rows.size, dtype=np.float64)
     for i, r in enumerate(rows):
         qr = _f64(q[b, h, r:r + 1])
-        o_r, l_r = attention_head(qr, kk, vv, scale, causal, row_offset=int(r), window_left=window_left)
+        keep = None if block_mask is None else block_keep(block_mask[b, h], [int(r)], kk.shape[0])
+        o_r, l_r = attention_head(qr, kk, vv, scale, causal, row_offset=int(r), window_left=window_left,
+                                  keep=keep)
         out_o[i] = o_r[0]
         out_l[i] = l_r[0]
     return out_o, out_l

@@ -470,6 +470,71 @@ def pin_fp8_attention(o):
     assert np.max(np.abs(lse - l2)) < 1e-12
 
 
+# -- block-sparse masks -----------------------------------------------------------
+
+def _block_case(seed, causal):
+    rng = _rng(seed)
+    B, Hq, Hkv, N, d = 1, 2, 1, 300, 4   # 3 blocks of 128 (the last one ragged)
+    q = _rand(rng, B, Hq, N, d)
+    k = _rand(rng, B, Hkv, N, d)
+    v = _rand(rng, B, Hkv, N, d)
+    bm = rng.random((B, Hq, 3, 3)) < 0.5
+    bm[0, 0, 1, :] = False            # query block 1 of head 0 sees nothing
+    bm[0, 1] = True
+    bm[0, 1, 2, 0] = False            # head 1: the last query block skips the first key block
+    return q, k, v, bm
+
+
+def pin_block_mask_sdpa(o):
+    """Block-sparse mask against PyTorch's fp64 SDPA with the mask expanded to
+    elements by hand (key j of row i kept iff block (i // 128, j // 128) is
+    set), causal or not; rows that see no key give O = 0 and LSE = -inf."""
+    for causal in (False, True):
+        q, k, v, bm = _block_case(40, causal)
+        out, lse = o.attention_forward(q, k, v, causal, 0.5, block_mask=bm)
+        N = q.shape[2]
+        for h in range(2):
+            blk = torch.arange(N) // 128                       # block of each row / key
+            allowed = torch.from_numpy(bm[0, h])[blk[:, None], blk[None, :]]
+            if causal:
+                allowed &= torch.arange(N)[None, :] <= torch.arange(N)[:, None]
+            rows = allowed.any(dim=1)
+            tq = torch.from_numpy(q[0, h])
+            tk = torch.from_numpy(k[0, 0])
+            tv = torch.from_numpy(v[0, 0])
+            ref = torch.nn.functional.scaled_dot_product_attention(tq[rows][None], tk[None], tv[None],
+                                                                    attn_mask=allowed[rows][None], scale=0.5)[0]
+            ref_lse = torch.logsumexp((0.5 * (tq @ tk.T)).masked_fill(~allowed, float("-inf")), -1)
+            assert np.max(np.abs(out[0, h][rows.numpy()] - ref.numpy())) < 1e-12
+            assert np.max(np.abs(lse[0, h][rows.numpy()] - ref_lse[rows].numpy())) < 1e-12
+            empty = ~rows.numpy()
+            if h == 0:
+                assert empty[128:256].all()
+            assert np.all(out[0, h][empty] == 0.0) and np.all(np.isneginf(lse[0, h][empty]))
+
+
+def pin_block_mask_brute(o):
+    """Scalar brute force for one row per query block, and an all-ones block
+    mask is no mask at all."""
+    q, k, v, bm = _block_case(41, True)
+    out, lse = o.attention_forward(q, k, v, True, 0.5, block_mask=bm)
+    for h in range(2):
+        for i in (5, 200, 299):
+            keys = [j for j in range(i + 1) if bm[0, h, i // 128, j // 128]]
+            if not keys:
+                assert np.all(out[0, h, i] == 0.0) and np.isneginf(lse[0, h, i])
+                continue
+            w = [math.exp(0.5 * math.fsum(q[0, h, i, c] * k[0, 0, j, c] for c in range(4))) for j in keys]
+            z = math.fsum(w)
+            for c in range(4):
+                assert abs(out[0, h, i, c] - math.fsum(wj * v[0, 0, j, c] for wj, j in zip(w, keys)) / z) < 1e-12
+            assert abs(lse[0, h, i] - math.log(z)) < 1e-12
+    full = np.ones_like(bm)
+    o1, l1 = o.attention_forward(q, k, v, True, 0.5, block_mask=full)
+    o2, l2 = o.attention_forward(q, k, v, True, 0.5)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
 ALL_PINS = [
     pin_rows_sum_to_one,
     pin_constant_v,
@@ -490,4 +555,6 @@ ALL_PINS = [
     pin_fp8_code_points,
     pin_fp8_matches_library,
     pin_fp8_attention,
+    pin_block_mask_sdpa,
+    pin_block_mask_brute,
 ]

@@ -77,12 +77,12 @@ def _fresh_oracle():
 
 def _mut_drop_scale(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
-        q, k, 1.0, causal, row_offset, window_left)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
+        q, k, 1.0, causal, row_offset, window_left, keep)
 
 
 def _mut_mask_includes_diagonal(m):
-    def scores(q, k, scale, causal, row_offset=0, window_left=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
         s = float(scale) * (np.asarray(q, float) @ np.asarray(k, float).T)
         if causal:
             rows = np.arange(row_offset, row_offset + s.shape[0])[:, None]
@@ -93,7 +93,7 @@ def _mut_mask_includes_diagonal(m):
 
 
 def _mut_mask_off_by_one_late(m):
-    def scores(q, k, scale, causal, row_offset=0, window_left=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
         s = float(scale) * (np.asarray(q, float) @ np.asarray(k, float).T)
         if causal:
             rows = np.arange(row_offset, row_offset + s.shape[0])[:, None]
@@ -105,12 +105,12 @@ def _mut_mask_off_by_one_late(m):
 
 def _mut_no_mask(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
-        q, k, scale, False, row_offset, window_left)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
+        q, k, scale, False, row_offset, window_left, keep)
 
 
 def _mut_transposed_scores(m):
-    def scores(q, k, scale, causal, row_offset=0, window_left=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
         q = np.asarray(q, float)
         k = np.asarray(k, float)
         s = float(scale) * (k @ q.T)
@@ -148,8 +148,8 @@ def _mut_softmax_wrong_axis(m):
 
 
 def _mut_pv_transposed(m):
-    def head(q, k, v, scale, causal, row_offset=0, window_left=None):
-        s = m.attention_scores(q, k, scale, causal, row_offset, window_left)
+    def head(q, k, v, scale, causal, row_offset=0, window_left=None, keep=None):
+        s = m.attention_scores(q, k, scale, causal, row_offset, window_left, keep)
         p, lse = m.softmax_with_lse(s)
         v = np.asarray(v, float)
         if p.shape[0] == p.shape[1]:
@@ -176,22 +176,22 @@ def _mut_page_no_table(m):
 
 def _mut_scale_squared(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
-        q, k, scale * scale, causal, row_offset, window_left)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
+        q, k, scale * scale, causal, row_offset, window_left, keep)
 
 
 def _mut_window_off_by_one(m):
     orig = m.attention_scores
-    def scores(q, k, scale, causal, row_offset=0, window_left=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
         w = None if window_left is None or window_left < 0 else window_left + 1
-        return orig(q, k, scale, causal, row_offset, w)
+        return orig(q, k, scale, causal, row_offset, w, keep)
     m.attention_scores = scores
 
 
 def _mut_window_ignored(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None: orig(
-        q, k, scale, causal, row_offset, None)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
+        q, k, scale, causal, row_offset, None, keep)
 
 
 def _mut_append_shifted(m):
@@ -217,8 +217,8 @@ def _mut_append_ignores_table(m):
 
 def _mut_prefill_no_offset(m):
     orig = m.attention_head
-    def head(q, k, v, scale, causal, row_offset=0, window_left=None):
-        return orig(q, k, v, scale, causal, 0, window_left)
+    def head(q, k, v, scale, causal, row_offset=0, window_left=None, keep=None):
+        return orig(q, k, v, scale, causal, 0, window_left, keep)
     m.attention_head = head
 
 
@@ -256,6 +256,28 @@ def _mut_fp8_v_descale_ignored(m):
         q8, k8, v8, qd, kd, 1.0, causal, scale, row_chunk)
 
 
+def _mut_block_mask_transposed(m):
+    orig = m.block_keep
+    def f(bm, rows, n_keys, block=128):
+        bm = np.asarray(bm, dtype=bool)
+        return orig(np.swapaxes(bm, -1, -2), rows, n_keys, block)
+    m.block_keep = f
+
+
+def _mut_block_mask_ignored(m):
+    m.block_keep = lambda bm, rows, n_keys, block=128: np.ones((len(np.atleast_1d(rows)), int(n_keys)), dtype=bool)
+
+
+def _mut_empty_rows_nan(m):
+    def f(s):
+        s = np.asarray(s, float)
+        mx = np.max(s, axis=-1, keepdims=True)
+        with np.errstate(all="ignore"):
+            lse = mx + np.log(np.sum(np.exp(s - mx), axis=-1, keepdims=True))
+            return np.exp(s - lse), lse[..., 0]
+    m.softmax_with_lse = f
+
+
 MUTANTS = [
     _mut_drop_scale,
     _mut_scale_squared,
@@ -278,6 +300,9 @@ MUTANTS = [
     _mut_fp8_bias8,
     _mut_fp8_no_subnormals,
     _mut_fp8_v_descale_ignored,
+    _mut_block_mask_transposed,
+    _mut_block_mask_ignored,
+    _mut_empty_rows_nan,
 ]
 
 
