@@ -53,6 +53,8 @@ SIGNATURES = {
     "paged_attn_decode_graph_launch": (_c_i, [_c_p, _c_p]),
     "paged_attn_decode_graph_destroy": (_c_i, [_c_p]),
     "attn_device_status": (_c_i, [_c_p, ctypes.POINTER(ctypes.c_uint)]),
+    "attn_fwd_block_sparse": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p,
+                                     ctypes.c_longlong, ctypes.c_longlong, _c_p]),
     "attn_fwd_fp8": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_f, _c_f, _c_f,
                             _c_p]),
     "paged_kv_append": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
@@ -432,4 +434,54 @@ def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool
                             d, int(bool(causal)), float(scale), float(q_descale), float(k_descale), float(v_descale),
                             _stream_handle(stream))
     _check(rc, "attn_fwd_fp8")
+    return out, lse
+
+
+def pack_block_mask(keep: torch.Tensor) -> torch.Tensor:
+    """Boolean block mask [B', H', q_blocks, k_blocks] (B' in {1, B}, H' in
+    {1, Hq}; block = 128 rows / keys) -> the uint64 rows attn_fwd_block_sparse
+    reads: bit j % 64 of word j / 64 set iff keep[..., j].  Returned as int64
+    words [B', H', q_blocks, ceil(k_blocks / 64)] on keep's device."""
+    if keep.dim() != 4:
+        raise ValueError("keep must be [B, H, q_blocks, k_blocks]")
+    nw = -(-keep.shape[-1] // 64)
+    pad = torch.zeros(*keep.shape[:-1], nw * 64, dtype=torch.int64, device=keep.device)
+    pad[..., : keep.shape[-1]] = keep.to(torch.int64)
+    bits = pad.view(*keep.shape[:-1], nw, 64)
+    weights = torch.ones(64, dtype=torch.int64, device=keep.device) << torch.arange(64, device=keep.device)
+    return (bits * weights).sum(-1)  # bit 63 wraps to the sign bit: the same 64 bits
+
+
+def attn_fwd_block_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, keep: torch.Tensor,
+                          causal: bool = True, scale: float | None = None, out: torch.Tensor | None = None,
+                          lse: torch.Tensor | None = None, stream=None):
+    """attn_fwd with a block-sparse mask: ``keep`` boolean [B or 1, Hq or 1,
+    ceil(N/128), ceil(N/128)] (1 = the 128x128 block is computed).  Rows
+    that see no key give O = 0, LSE = -inf."""
+    _require(q, "q", torch.bfloat16, 4)
+    _require(k, "k", torch.bfloat16, 4)
+    _require(v, "v", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} do not match q {tuple(q.shape)}")
+    nb = -(-N // 128)
+    if keep.dim() != 4 or keep.shape[2:] != (nb, nb) or keep.shape[0] not in (1, B) or keep.shape[1] not in (1, Hq):
+        raise ValueError(f"keep must be [1 or {B}, 1 or {Hq}, {nb}, {nb}], got {tuple(keep.shape)}")
+    words = pack_block_mask(keep.to(q.device)).contiguous()
+    nw = words.shape[-1]
+    h_stride = 0 if keep.shape[1] == 1 else nb * nw
+    b_stride = 0 if keep.shape[0] == 1 else keep.shape[1] * nb * nw
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _require(out, "out", torch.bfloat16, 4)
+    _require(lse, "lse", torch.float32, 3)
+    rc = lib().attn_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq,
+                                     Hkv, N, d, int(bool(causal)), float(scale), words.data_ptr(), b_stride, h_stride,
+                                     _stream_handle(stream))
+    _check(rc, "attn_fwd_block_sparse")
     return out, lse

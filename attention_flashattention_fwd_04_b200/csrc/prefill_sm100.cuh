@@ -86,7 +86,15 @@ struct PrefillParams {
   const __nv_bfloat16* v_pool;
   int num_seqs, total_q, max_pages, num_pages, page_size;
   int page_box;                // rows per K/V TMA box: min(page_size, 128)
+  // Block-sparse (kernels with SPARSE only): bit j % 64 of word j / 64 of row
+  // qb of head (b, h) keeps KV tile j for query tile qb; rows of mask_words
+  // words at block_mask + b * mask_b_stride + h * mask_h_stride + qb * mask_words.
+  const uint64_t* block_mask;
+  long long mask_b_stride, mask_h_stride;
+  int mask_words;              // ceil(ceil(N / 128) / 64), at most kMaskWords
 };
+
+constexpr int kMaskWords = 4;  // block-sparse masks cover N <= 4 * 64 * 128 = 32768
 
 constexpr int kPagedMaxSeqs = 1024;    // sequences per paged-prefill call
 constexpr int kPagedMaxBlocks = 2048;  // 256-row query blocks per paged-prefill call
@@ -100,7 +108,7 @@ constexpr float kFp8PLog2 = 8.0f;
 constexpr float kRescaleThresholdFp8 = 0.5f;
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D, bool PAGED = false, bool FP8 = false>
+template <int D, bool PAGED = false, bool FP8 = false, bool SPARSE = false>
 struct PrefillLayout {
   static_assert(!FP8 || D == 128, "FP8 tiles are one 128-byte box wide");
   static constexpr int NS = 2;                     // K and V ring depth
@@ -118,8 +126,16 @@ struct PrefillLayout {
   // Paged: cached at kernel start: the query blocks in processing order
   // [kPagedMaxBlocks], cu_q [S+1], seq_lens [S], the block count and 16 ints
   // of scan scratch.
+  // Block-sparse: the current item's KV-tile sets, as words in shared memory
+  // (read back on use, so the loops hold none in registers): the MMA
+  // thread's both sets, the producer's union, one query tile's set per
+  // softmax warp.
   static constexpr int kSeq = kStats + kStatsBytes;
-  static constexpr int kSeqBytes = PAGED ? (kPagedMaxBlocks + 2 * kPagedMaxSeqs + 1 + 1 + 16) * 4 : 0;
+  // The MMA thread also lists the item's tiles (16-bit entries, up to 256).
+  static constexpr int kMaskMma = 0, kMaskProd = 8, kMaskSoftmax = 12;  // in words, from kSeq
+  static constexpr int kTileList = (8 + 4 + 8 * 4) * 8;                  // bytes, from kSeq
+  static constexpr int kSeqBytes = PAGED ? (kPagedMaxBlocks + 2 * kPagedMaxSeqs + 1 + 1 + 16) * 4
+                                         : SPARSE ? kTileList + 64 * kMaskWords * 2 : 0;
   static constexpr int kBar = (kSeq + kSeqBytes + 7) / 8 * 8;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarQEmpty = 1;
@@ -152,11 +168,60 @@ struct PrefillItem {
   int lo0, hi0, lo1, hi1;  // tile 1 is empty (lo1 = hi1) when its rows lie past N
   int jb, je;
   int q0, n_q, n_kv, pos0;  // paged only
+  // Block-sparse only: the KV tiles each query tile visits, as bits (tile j:
+  // bit j % 64 of word j / 64), already limited to [lo, hi).
+  uint64_t mk0[kMaskWords], mk1[kMaskWords];
   __device__ __forceinline__ int lo(int t) const { return t ? lo1 : lo0; }
   __device__ __forceinline__ int hi(int t) const { return t ? hi1 : hi0; }
   __device__ __forceinline__ bool active(int t, int j) const { return lo(t) <= j && j < hi(t); }
   __device__ __forceinline__ bool has(int t) const { return hi(t) > lo(t); }
 };
+
+// Bits [lo, hi) of a 64-bit word (0 <= lo, hi <= 64).
+__device__ __forceinline__ uint64_t bit_range(int lo, int hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 64);
+  if (hi <= lo) return 0ull;
+  const uint64_t upto = hi == 64 ? ~0ull : ((1ull << hi) - 1ull);
+  return upto & (~0ull << lo);
+}
+
+// Smallest set bit above j in a 4-word set, or 64 * kMaskWords if none.
+__device__ __forceinline__ int next_bit(uint64_t w0, uint64_t w1, uint64_t w2, uint64_t w3, int j) {
+  const int from = j + 1;
+#pragma unroll
+  for (int k = 0; k < kMaskWords; ++k) {
+    uint64_t w = k == 0 ? w0 : k == 1 ? w1 : k == 2 ? w2 : w3;
+    const int lo_bit = from - k * 64;
+    if (lo_bit >= 64) continue;
+    if (lo_bit > 0) w &= ~0ull << lo_bit;
+    if (w) return k * 64 + __ffsll(static_cast<long long>(w)) - 1;
+  }
+  return 64 * kMaskWords;
+}
+
+// The same over four words in shared memory (read when needed).
+__device__ __forceinline__ int next_bit_s(const volatile uint64_t* w, int j) {
+  return next_bit(w[0], w[1], w[2], w[3], j);
+}
+__device__ __forceinline__ int next_bit_union_s(const volatile uint64_t* a, const volatile uint64_t* b, int j) {
+  return next_bit(a[0] | b[0], a[1] | b[1], a[2] | b[2], a[3] | b[3], j);
+}
+__device__ __forceinline__ bool bit_s(const volatile uint64_t* w, int j) {
+  return j >= 0 && j < 64 * kMaskWords && ((w[j >> 6] >> (j & 63)) & 1ull) != 0ull;
+}
+// Number of KV tiles query tile t of an item visits (block-sparse: its set's size).
+template <bool SPARSE>
+__device__ __forceinline__ int tile_count(const PrefillItem& it, int t) {
+  if constexpr (SPARSE) {
+    int n = 0;
+#pragma unroll
+    for (int k = 0; k < kMaskWords; ++k) n += __popcll(t ? it.mk1[k] : it.mk0[k]);
+    return n;
+  } else {
+    return it.hi(t) - it.lo(t);
+  }
+}
 
 // Sequence table of the paged kernels, in shared memory.
 struct PagedSeqs {
@@ -208,7 +273,7 @@ __device__ __forceinline__ bool paged_item(int idx, const PrefillParams& p, cons
   return true;
 }
 
-template <bool CAUSAL, bool WINDOW, bool PAGED = false>
+template <bool CAUSAL, bool WINDOW, bool PAGED = false, bool SPARSE = false>
 __device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, PrefillItem& it,
                                              const PagedSeqs& sq = PagedSeqs{}) {
   const int G = static_cast<int>(gridDim.x);
@@ -244,6 +309,20 @@ __device__ __forceinline__ bool prefill_item(int round, const PrefillParams& p, 
   }
   it.jb = it.lo0;
   it.je = max(it.hi0, it.has(1) ? it.hi1 : 0);
+  if constexpr (SPARSE) {
+    const uint64_t* rows = p.block_mask + it.b * p.mask_b_stride + it.h * p.mask_h_stride;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const uint64_t* row = rows + static_cast<long long>(2 * it.m + t) * p.mask_words;
+      const bool live = it.has(t);
+#pragma unroll
+      for (int k = 0; k < kMaskWords; ++k) {
+        const uint64_t w = (live && k < p.mask_words) ? row[k] : 0ull;
+        const uint64_t keep = w & bit_range(it.lo(t) - 64 * k, it.hi(t) - 64 * k);
+        if (t) it.mk1[k] = keep; else it.mk0[k] = keep;
+      }
+    }
+  }
   return true;
 }
 
@@ -368,7 +447,7 @@ __device__ __forceinline__ void reg_alloc_control() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
 }
 
-template <int D, bool CAUSAL, bool WINDOW, bool PAGED, bool FP8 = false>
+template <int D, bool CAUSAL, bool WINDOW, bool PAGED, bool FP8 = false, bool SPARSE = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -376,7 +455,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(!(PAGED && WINDOW), "the paged kernels have no window");
   static_assert(!(FP8 && (PAGED || WINDOW)), "the FP8 kernels are dense, without a window");
-  using L = PrefillLayout<D, PAGED, FP8>;
+  static_assert(!(SPARSE && (PAGED || WINDOW || FP8)), "the block-sparse kernels are dense bf16");
+  using L = PrefillLayout<D, PAGED, FP8, SPARSE>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -384,6 +464,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* smem = smem_raw + (base - raw);
   auto bar = [&](int i) -> uint32_t { return base + L::kBar + 8u * static_cast<uint32_t>(i); };
   float* stats = reinterpret_cast<float*>(smem + L::kStats);
+  // Block-sparse mask words (SPARSE only), see PrefillLayout.
+  volatile uint64_t* const mask_smem = reinterpret_cast<volatile uint64_t*>(smem + L::kSeq);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -559,7 +641,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ++v_issued;
         return true;
       };
-      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
+      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
         // Q rows: dense (d, row, b*Hq + h); paged (d, packed token, h).
         const int qz = PAGED ? it.h : it.b * p.Hq + it.h;
         const int qrow = (PAGED ? it.q0 : 0) + it.m * 256;
@@ -568,10 +650,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tile_j = -1;  // a new item: its own sequence, pages and table row
         win_base = -(1 << 30);
         have_next = false;
+        // Block-sparse: the item's union of sets, in shared memory for the warp.
+        volatile uint64_t* const mu = mask_smem + L::kMaskProd;
+        if constexpr (SPARSE) {
+          __syncwarp();
+          if (lane == 0) {
+#pragma unroll
+            for (int k = 0; k < kMaskWords; ++k) mu[k] = it.mk0[k] | it.mk1[k];
+          }
+          __syncwarp();
+        }
+        auto unext = [&](int j) { return SPARSE ? min(next_bit_s(mu, j), it.je) : j + 1; };
+        const int j0 = SPARSE ? unext(it.jb - 1) : it.jb;
+        if (j0 >= it.je) continue;  // block-sparse: every tile of the item masked, nothing to load
         // The item's first K tile first: it can land while the previous item
         // still holds Q.
-        if (!(ok = load_k(it.jb, kz))) break;
-        if (r > 0 && !(ok = wait0(bar(L::kBarQEmpty), static_cast<uint32_t>(r - 1) & 1u, kErrWaitQ))) break;
+        if (!(ok = load_k(j0, kz))) break;
+        if (q_issued > 0 &&
+            !(ok = wait0(bar(L::kBarQEmpty), static_cast<uint32_t>(q_issued - 1) & 1u, kErrWaitQ)))
+          break;
         if (lane == 0) {
           mbar_arrive_expect_tx(bar(L::kBarQFull), (it.has(1) ? 2 : 1) * L::kTileBytes);
           for (int c = 0; c < L::kBoxes; ++c)
@@ -582,9 +679,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                           qz);
         }
         ++q_issued;
-        if (!(ok = load_v(it.jb, kz))) break;
+        if (!(ok = load_v(j0, kz))) break;
         ++kv_it;
-        for (int j = it.jb + 1; j < it.je; ++j, ++kv_it) {
+        for (int j = unext(j0); j < it.je; j = unext(j), ++kv_it) {
           if (!(ok = load_k(j, kz))) break;
           if (!(ok = load_v(j, kz))) break;
         }
@@ -643,71 +740,183 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       };
       PrefillItem it;
-      for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
-        if (!(ok = mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(r) & 1u, kErrWaitQ))) break;
-        const int nkv = it.je - it.jb;
-        {
-          const int st = kv_it % NS;
-          if (!(ok = mbar_wait(bar(L::kBarKFull + st), static_cast<uint32_t>(kv_it / NS) & 1u, kErrWaitKFull)))
-            break;
-          tc_fence_after();
-          if (it.active(0, it.jb)) issue_s(0, st);
-          if (it.active(1, it.jb)) issue_s(1, st);
-          mma_commit(bar(L::kBarKEmpty + st));
-          if (nkv == 1) mma_commit(bar(L::kBarQEmpty));  // last S of the item: Q may be replaced
-        }
-        for (int j = it.jb; j < it.je && ok; ++j) {
-          const int g = kv_it + (j - it.jb);
-          const int st = g % NS, st1 = (g + 1) % NS;
-          const uint32_t ph = static_cast<uint32_t>(g / NS) & 1u, ph1 = static_cast<uint32_t>((g + 1) / NS) & 1u;
-          bool v_ready = false, k_ready = false;
-          if (it.active(0, j)) {
-            const uint32_t pph = p_cnt[0]++ & 1u;
-            if (!(ok = mbar_wait(bar(L::kBarPFull + 0), pph, kErrWaitPFull))) break;
-            if (j == it.lo0 && o_cnt[0] > 0 &&
-                !(ok = mbar_wait(bar(L::kBarOFree + 0), (o_cnt[0] - 1u) & 1u, kErrWaitODone)))
-              break;
-            if (!(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
-            v_ready = true;
-            tc_fence_after();
-            issue_pv(0, st, j > it.lo0);
-            if (j + 1 == it.hi0) {
-              mma_commit(bar(L::kBarOFull + 0));  // O0 of this item is final once this lands
-              ++o_cnt[0];
+      if constexpr (SPARSE) {
+        // Block-sparse: each query tile visits an arbitrary set of KV tiles;
+        // the item walks their union.
+        uint32_t q_cnt = 0;  // items whose Q was loaded (every item except fully masked block-sparse ones)
+        for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
+          // This thread's copy of the item's two sets (shared memory, re-read on use).
+          volatile uint64_t* const mm0 = mask_smem + L::kMaskMma;
+          volatile uint64_t* const mm1 = mm0 + kMaskWords;
+#pragma unroll
+          for (int k = 0; k < kMaskWords; ++k) {
+            mm0[k] = it.mk0[k];
+            mm1[k] = it.mk1[k];
+          }
+          // The item's tiles in order, one 16-bit entry each: tile index (bits
+          // 0-7), visited by query tile 0 / 1 (bits 8, 9), first for it
+          // (10, 11), last for it (12, 13).  Listed while Q is in flight.
+          volatile uint16_t* const tl = reinterpret_cast<volatile uint16_t*>(smem + L::kSeq + L::kTileList);
+          int n_u = 0;
+          {
+            int seen0 = 0, seen1 = 0;
+            for (int j = next_bit_union_s(mm0, mm1, it.jb - 1); j < it.je; j = next_bit_union_s(mm0, mm1, j)) {
+              const int a = bit_s(mm0, j), b = bit_s(mm1, j);
+              int e = j | (a << 8) | (b << 9);
+              if (a && !seen0) e |= 1 << 10;
+              if (b && !seen1) e |= 1 << 11;
+              if (a && next_bit_s(mm0, j) >= 64 * kMaskWords) e |= 1 << 12;
+              if (b && next_bit_s(mm1, j) >= 64 * kMaskWords) e |= 1 << 13;
+              seen0 |= a;
+              seen1 |= b;
+              tl[n_u++] = static_cast<uint16_t>(e);
             }
-            if (it.active(0, j + 1)) {
+          }
+          if (n_u == 0) continue;  // nothing to compute (the epilogue writes zeros)
+          auto on = [&](int t, int e) { return ((e >> (8 + t)) & 1) != 0; };
+          if (!(ok = mbar_wait(bar(L::kBarQFull), q_cnt & 1u, kErrWaitQ))) break;
+          ++q_cnt;
+          {
+            const int st = kv_it % NS;
+            if (!(ok = mbar_wait(bar(L::kBarKFull + st), static_cast<uint32_t>(kv_it / NS) & 1u, kErrWaitKFull)))
+              break;
+            tc_fence_after();
+            if (on(0, tl[0])) issue_s(0, st);
+            if (on(1, tl[0])) issue_s(1, st);
+            mma_commit(bar(L::kBarKEmpty + st));
+            if (n_u == 1) mma_commit(bar(L::kBarQEmpty));  // last S of the item
+          }
+          // First and last KV tile of each query tile: where O_t starts (after
+          // the epilogue released it) and where it is final.
+          auto first_of = [&](int t, int e) { return ((e >> (10 + t)) & 1) != 0; };
+          auto last_of = [&](int t, int e) { return ((e >> (12 + t)) & 1) != 0; };
+          int u = 0;  // position among the item's tiles (K/V ring slot kv_it + u)
+          for (; u < n_u && ok; ++u) {
+            const int e = tl[u];                        // this tile
+            const bool more = u + 1 < n_u;
+            const int en = more ? tl[u + 1] : 0;        // the next one
+            const int g = kv_it + u;
+            const int st = g % NS, st1 = (g + 1) % NS;
+            const uint32_t ph = static_cast<uint32_t>(g / NS) & 1u, ph1 = static_cast<uint32_t>((g + 1) / NS) & 1u;
+            bool v_ready = false, k_ready = false;
+            if (on(0, e)) {
+              const uint32_t pph = p_cnt[0]++ & 1u;
+              if (!(ok = mbar_wait(bar(L::kBarPFull + 0), pph, kErrWaitPFull))) break;
+              if (first_of(0, e) && o_cnt[0] > 0 &&
+                  !(ok = mbar_wait(bar(L::kBarOFree + 0), (o_cnt[0] - 1u) & 1u, kErrWaitODone)))
+                break;
+              if (!(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
+              v_ready = true;
+              tc_fence_after();
+              issue_pv(0, st, !first_of(0, e));
+              if (last_of(0, e)) {
+                mma_commit(bar(L::kBarOFull + 0));  // O0 of this item is final once this lands
+                ++o_cnt[0];
+              }
+            }
+            if (more && on(0, en)) {
+              // Q0's next S.  P0, which S0 overwrites, went into a P V already
+              // issued (this tile's or an earlier one's).
               if (!(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
               k_ready = true;
               tc_fence_after();
               issue_s(0, st1);
             }
-          }
-          if (it.active(1, j)) {
-            const uint32_t pph = p_cnt[1]++ & 1u;
-            if (!(ok = mbar_wait(bar(L::kBarPFull + 1), pph, kErrWaitPFull))) break;
-            if (j == it.lo1 && o_cnt[1] > 0 &&
-                !(ok = mbar_wait(bar(L::kBarOFree + 1), (o_cnt[1] - 1u) & 1u, kErrWaitODone)))
-              break;
-            if (!v_ready && !(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
-            tc_fence_after();
-            issue_pv(1, st, j > it.lo1);
-            if (j + 1 == it.hi1) {
-              mma_commit(bar(L::kBarOFull + 1));
-              ++o_cnt[1];
+            if (on(1, e)) {
+              const uint32_t pph = p_cnt[1]++ & 1u;
+              if (!(ok = mbar_wait(bar(L::kBarPFull + 1), pph, kErrWaitPFull))) break;
+              if (first_of(1, e) && o_cnt[1] > 0 &&
+                  !(ok = mbar_wait(bar(L::kBarOFree + 1), (o_cnt[1] - 1u) & 1u, kErrWaitODone)))
+                break;
+              if (!v_ready && !(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
+              tc_fence_after();
+              issue_pv(1, st, !first_of(1, e));
+              if (last_of(1, e)) {
+                mma_commit(bar(L::kBarOFull + 1));
+                ++o_cnt[1];
+              }
             }
+            if (more && on(1, en)) {
+              // Q1's next S; also its first one when its range starts at jn.
+              if (!k_ready && !(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
+              tc_fence_after();
+              issue_s(1, st1);
+            }
+            mma_commit(bar(L::kBarVEmpty + st));
+            if (more) mma_commit(bar(L::kBarKEmpty + st1));
+            if (u + 2 == n_u) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
           }
-          if (it.active(1, j + 1)) {
-            // Q1's next S; also its first one when its window starts at j + 1.
-            if (!k_ready && !(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
-            tc_fence_after();
-            issue_s(1, st1);
-          }
-          mma_commit(bar(L::kBarVEmpty + st));
-          if (j + 1 < it.je) mma_commit(bar(L::kBarKEmpty + st1));
-          if (j + 2 == it.je) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
+          if (!ok) break;
+          kv_it += u;
         }
-        if (!ok) break;
-        kv_it += nkv;
+      } else {
+        // Dense: query tile t visits the contiguous range [lo(t), hi(t)).
+        for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
+          if (!(ok = mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(r) & 1u, kErrWaitQ))) break;
+          const int nkv = it.je - it.jb;
+          {
+            const int st = kv_it % NS;
+            if (!(ok = mbar_wait(bar(L::kBarKFull + st), static_cast<uint32_t>(kv_it / NS) & 1u, kErrWaitKFull)))
+              break;
+            tc_fence_after();
+            if (it.active(0, it.jb)) issue_s(0, st);
+            if (it.active(1, it.jb)) issue_s(1, st);
+            mma_commit(bar(L::kBarKEmpty + st));
+            if (nkv == 1) mma_commit(bar(L::kBarQEmpty));  // last S of the item: Q may be replaced
+          }
+          for (int j = it.jb; j < it.je && ok; ++j) {
+            const int g = kv_it + (j - it.jb);
+            const int st = g % NS, st1 = (g + 1) % NS;
+            const uint32_t ph = static_cast<uint32_t>(g / NS) & 1u, ph1 = static_cast<uint32_t>((g + 1) / NS) & 1u;
+            bool v_ready = false, k_ready = false;
+            if (it.active(0, j)) {
+              const uint32_t pph = p_cnt[0]++ & 1u;
+              if (!(ok = mbar_wait(bar(L::kBarPFull + 0), pph, kErrWaitPFull))) break;
+              if (j == it.lo0 && o_cnt[0] > 0 &&
+                  !(ok = mbar_wait(bar(L::kBarOFree + 0), (o_cnt[0] - 1u) & 1u, kErrWaitODone)))
+                break;
+              if (!(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
+              v_ready = true;
+              tc_fence_after();
+              issue_pv(0, st, j > it.lo0);
+              if (j + 1 == it.hi0) {
+                mma_commit(bar(L::kBarOFull + 0));  // O0 of this item is final once this lands
+                ++o_cnt[0];
+              }
+              if (it.active(0, j + 1)) {
+                if (!(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
+                k_ready = true;
+                tc_fence_after();
+                issue_s(0, st1);
+              }
+            }
+            if (it.active(1, j)) {
+              const uint32_t pph = p_cnt[1]++ & 1u;
+              if (!(ok = mbar_wait(bar(L::kBarPFull + 1), pph, kErrWaitPFull))) break;
+              if (j == it.lo1 && o_cnt[1] > 0 &&
+                  !(ok = mbar_wait(bar(L::kBarOFree + 1), (o_cnt[1] - 1u) & 1u, kErrWaitODone)))
+                break;
+              if (!v_ready && !(ok = mbar_wait(bar(L::kBarVFull + st), ph, kErrWaitVFull))) break;
+              tc_fence_after();
+              issue_pv(1, st, j > it.lo1);
+              if (j + 1 == it.hi1) {
+                mma_commit(bar(L::kBarOFull + 1));
+                ++o_cnt[1];
+              }
+            }
+            if (it.active(1, j + 1)) {
+              // Q1's next S; also its first one when its window starts at j + 1.
+              if (!k_ready && !(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
+              tc_fence_after();
+              issue_s(1, st1);
+            }
+            mma_commit(bar(L::kBarVEmpty + st));
+            if (j + 1 < it.je) mma_commit(bar(L::kBarKEmpty + st1));
+            if (j + 2 == it.je) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
+          }
+          if (!ok) break;
+          kv_it += nkv;
+        }
       }
       // All issued MMAs must finish before tensor memory is released.
       mma_commit(bar(L::kBarMmaDone));
@@ -722,10 +931,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t st_cnt[2] = {0u, 0u};  // items whose tile t this warpgroup has written out
     bool ok = true;
     PrefillItem it;
-    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
+    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (!it.has(t)) continue;
+        if constexpr (SPARSE) {
+          if (tile_count<SPARSE>(it, t) == 0) {
+            // Every KV tile of this query tile is masked: its rows see no key,
+            // O = 0 and LSE = -inf, with nothing computed to wait for.
+            const int grow = it.m * 256 + t * 128 + row;
+            if (grow < p.N) {
+              const size_t row_index = static_cast<size_t>(it.b * p.Hq + it.h) * p.N + grow;
+              uint4* dst = reinterpret_cast<uint4*>(p.o + row_index * D);
+#pragma unroll
+              for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+              p.lse[row_index] = -INFINITY;
+            }
+            continue;
+          }
+        }
         const uint32_t n = st_cnt[t];
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarOFull + t), n & 1u, kErrWaitODone));
         if (!ok) break;
@@ -779,9 +1003,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t s_cnt = 0, st_cnt = 0;
     bool ok = true;
     PrefillItem it;
-    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED>(r, p, it, sq); ++r) {
-      const int lo_t = it.lo(t);
-      const int n_t = it.hi(t) - lo_t;  // KV tiles this query tile visits (>= 0)
+    for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
+      // Block-sparse: this query tile's set, in this warp's shared-memory slot.
+      volatile uint64_t* const mw = mask_smem + L::kMaskSoftmax + warp * kMaskWords;
+      if constexpr (SPARSE) {
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int k = 0; k < kMaskWords; ++k) mw[k] = t ? it.mk1[k] : it.mk0[k];
+        }
+        __syncwarp();
+      }
+      const int lo_t = SPARSE ? next_bit_s(mw, -1) : it.lo(t);
+      // KV tiles it visits (>= 0); block-sparse: 1 when the set is not empty
+      // (its loop ends on the set's last tile instead).
+      const int n_t = SPARSE ? (lo_t < 64 * kMaskWords ? 1 : 0) : it.hi(t) - lo_t;
       if (n_t == 0) continue;
       // Position (key index) of this tile's first query row; paged chunks
       // start at the sequence's cached length.
@@ -790,8 +1026,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int n_kv = PAGED ? it.n_kv : p.N;
       float m_used = -INFINITY;  // running max in scaled log2 units
       float l_sum = 0.f;
-      for (int jj = 0; jj < n_t; ++jj) {
-        const int j = lo_t + jj;
+      int j_set = lo_t - 1;  // block-sparse: the previous tile of this query tile's set
+      for (int jj = 0; SPARSE ? next_bit_s(mw, j_set) < 64 * kMaskWords : jj < n_t; ++jj) {
+        const int j = SPARSE ? (j_set = next_bit_s(mw, j_set)) : lo_t + jj;
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarSFull + t), s_cnt++ & 1u, kErrWaitSFull));
         if (!ok) break;
         tc_fence_after();

@@ -100,6 +100,24 @@ int attn_fwd_window(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, 
                     float scale, void* stream);
 
 /*
+ * attn_fwd_block_sparse -- attn_fwd with a 2-D block-sparse mask (the
+ * block-sparse masks of FlashInfer, e.g. Longformer's window-plus-global
+ * pattern, "Kernel Fusion and Custom Kernels", ai.zenoagi.com, section 4):
+ * key j is visible to query i only if block (i / 128, j / 128) is kept, on top
+ * of the causal mask.  KV tiles of masked blocks are never loaded or computed.
+ *   block_mask: uint64 words; query block qb of head (b, h) keeps KV block j
+ *   iff bit j % 64 of word j / 64 is set in the row of ceil(ceil(N/128)/64)
+ *   words at block_mask + b * mask_b_stride + h * mask_h_stride
+ *   + qb * ceil(ceil(N/128)/64) (strides in words; 0 broadcasts; 8-byte
+ *   aligned; bits past the last KV block are ignored).
+ * A query row that sees no key at all gets O = 0 and LSE = -inf.  N <= 32768
+ * (ATTN_ERR_UNSUPPORTED above).  Other arguments and errors as attn_fwd.
+ */
+int attn_fwd_block_sparse(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse,
+                          int B, int Hq, int Hkv, int N, int d, int causal, float scale, const uint64_t* block_mask,
+                          long long mask_b_stride, long long mask_h_stride, void* stream);
+
+/*
  * attn_fwd_fp8 -- attn_fwd with e4m3 inputs (OCP FP8 E4M3 codes, one byte
  * each, same [B, H, N, d] layouts): the attention of q * q_descale,
  * k * k_descale and v * v_descale, the FP8 tensor-core path of FlashAttention

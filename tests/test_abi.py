@@ -188,3 +188,19 @@ def _fp8(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=16, 
 ])
 def test_attn_fwd_fp8_rejects(lib, kw, code):
     assert _fp8(lib, **kw) == code
+
+
+def _bs(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=300, d=128, causal=1, scale=0.1,
+        mask=FAKE, bs=0, hs=0):
+    return lib.attn_fwd_block_sparse(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, mask, bs, hs, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(mask=None), 1), (dict(q=None), 1),
+    (dict(N=0), 2), (dict(d=96), 2), (dict(causal=2), 2), (dict(scale=0.0), 2), (dict(bs=-1), 2),
+    (dict(hs=-5), 2),
+    (dict(N=32769), 5),
+    (dict(mask=FAKE + 4), 3), (dict(q=FAKE + 8), 3),
+])
+def test_attn_fwd_block_sparse_rejects(lib, kw, code):
+    assert _bs(lib, **kw) == code
