@@ -41,6 +41,9 @@ Readings where the pages are silent (each is restated where it is used):
   masked 128 x 128 block, on top of the causal mask.  A row that sees no key
   at all outputs zeros with LSE = -inf (the pages leave it open; this is the
   decode's convention for an empty sequence).
+* additive M (the attention equation's M in general: any finite values, -inf
+  allowed): a [B|1, Hq|1, N, N] array in natural-log units added to the
+  scaled scores, S = scale * q k^T + M, on top of the causal mask.
 * FP8 inputs (the anylearn.cc lesson's FA v3 section: Q K^T and P V computed
   in FP8): Q, K, V arrive as e4m3 codes with one descale factor per tensor;
   the operation is attention over the decoded values times their descales
@@ -107,7 +110,7 @@ def gqa_kv_head(h_q: int, Hq: int, Hkv: int) -> int:
 
 
 def attention_scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
-                     row_offset: int = 0, window_left: int | None = None, keep=None) -> np.ndarray:
+                     row_offset: int = 0, window_left: int | None = None, keep=None, bias=None) -> np.ndarray:
     """S = scale * q k^T + M for one head.
 
     ``q`` holds query rows ``row_offset .. row_offset + len(q) - 1`` of the head;
@@ -120,6 +123,8 @@ def attention_scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
     q = _f64(q)
     k = _f64(k)
     s = float(scale) * (q @ k.T)
+    if bias is not None:  # additive M, [len(q), len(k)]
+        s = s + _f64(bias)
     rows = np.arange(row_offset, row_offset + q.shape[0])[:, None]
     cols = np.arange(k.shape[0])[None, :]
     if causal:
@@ -149,9 +154,9 @@ def softmax_with_lse(s: np.ndarray):
 
 
 def attention_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float,
-                   causal: bool, row_offset: int = 0, window_left: int | None = None, keep=None):
+                   causal: bool, row_offset: int = 0, window_left: int | None = None, keep=None, bias=None):
     """O and LSE for one head: materialise S, then P, then O = P V."""
-    s = attention_scores(q, k, scale, causal, row_offset, window_left, keep)
+    s = attention_scores(q, k, scale, causal, row_offset, window_left, keep, bias)
     p, lse = softmax_with_lse(s)
     o = p @ _f64(v)
     return o, lse
@@ -168,13 +173,14 @@ def block_keep(block_mask_bh, rows, n_keys: int, block: int = 128) -> np.ndarray
 
 
 def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None = None,
-                      window_left: int | None = None, block_mask=None):
+                      window_left: int | None = None, block_mask=None, bias=None):
     """Full attention forward for [B, Hq, N, d] queries and [B, Hkv, N, d] K/V.
 
     Returns (O [B, Hq, N, d] float64, LSE [B, Hq, N] float64).  ``row_chunk``
     splits each head into blocks of complete query rows (every row still sees
     its whole key set), which only bounds memory for long sequences.
     ``block_mask``: boolean [B, Hq, ceil(N/128), ceil(N/128)] (see block_keep).
+    ``bias``: additive M, [B or 1, Hq or 1, N, N], natural-log units.
     """
     q = _f64(q)
     k = _f64(k)
@@ -190,14 +196,18 @@ def attention_forward(q, k, v, causal: bool, scale: float, row_chunk: int | None
             for r0 in range(0, N, step):
                 r1 = min(N, r0 + step)
                 keep = None if block_mask is None else block_keep(block_mask[b, h], np.arange(r0, r1), N)
+                mb = None
+                if bias is not None:
+                    bb = np.asarray(bias)
+                    mb = bb[b if bb.shape[0] > 1 else 0, h if bb.shape[1] > 1 else 0, r0:r1]
                 o[b, h, r0:r1], lse[b, h, r0:r1] = attention_head(
                     q[b, h, r0:r1], k[b, hk], v[b, hk], scale, causal, row_offset=r0,
-                    window_left=window_left, keep=keep)
+                    window_left=window_left, keep=keep, bias=mb)
     return o, lse
 
 
 def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows,
-                   window_left: int | None = None, block_mask=None):
+                   window_left: int | None = None, block_mask=None, bias=None):
     """O and LSE of selected query rows of head (b, h), each row exact.
 
     Used for sampled parity checks at sizes where the full oracle is too slow.
@@ -212,8 +222,12 @@ def attention_rows(q, k, v, causal: bool, scale: float, b: int, h: int, rows,
     for i, r in enumerate(rows):
         qr = _f64(q[b, h, r:r + 1])
         keep = None if block_mask is None else block_keep(block_mask[b, h], [int(r)], kk.shape[0])
+        mb = None
+        if bias is not None:
+            bb = np.asarray(bias)
+            mb = bb[b if bb.shape[0] > 1 else 0, h if bb.shape[1] > 1 else 0, int(r):int(r) + 1]
         o_r, l_r = attention_head(qr, kk, vv, scale, causal, row_offset=int(r), window_left=window_left,
-                                  keep=keep)
+                                  keep=keep, bias=mb)
         out_o[i] = o_r[0]
         out_l[i] = l_r[0]
     return out_o, out_l

@@ -535,6 +535,61 @@ def pin_block_mask_brute(o):
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
+# -- additive M ---------------------------------------------------------------------
+
+def pin_bias_sdpa(o):
+    """Additive M against PyTorch's fp64 SDPA with a float attn_mask (which is
+    added to the scaled scores) and logsumexp of the biased scores, with a
+    broadcast over batch and per-head M, causal or not; -inf entries allowed."""
+    rng = _rng(50)
+    B, Hq, Hkv, N, d = 2, 2, 1, 37, 8
+    q = _rand(rng, B, Hq, N, d)
+    k = _rand(rng, B, Hkv, N, d)
+    v = _rand(rng, B, Hkv, N, d)
+    m = rng.standard_normal((1, Hq, N, N)) * 2.0
+    m[0, 1, :, :3] = -np.inf                       # head 1: the first three keys masked by M
+    m[0, 1, :3, 3:] = 0.0
+    for causal in (False, True):
+        out, lse = o.attention_forward(q, k, v, causal, 0.3, bias=m)
+        for b in range(B):
+            for h in range(Hq):
+                tm = torch.from_numpy(m[0, h].copy())
+                if causal:
+                    tm = tm.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+                tq, tk, tv = (torch.from_numpy(x) for x in (q[b, h], k[b, 0], v[b, 0]))
+                rows = torch.isfinite(tm).any(dim=1)
+                ref = torch.nn.functional.scaled_dot_product_attention(tq[rows][None], tk[None], tv[None],
+                                                                        attn_mask=tm[rows][None], scale=0.3)[0]
+                ref_lse = torch.logsumexp(0.3 * (tq @ tk.T) + tm, -1)
+                assert np.max(np.abs(out[b, h][rows.numpy()] - ref.numpy())) < 1e-12
+                assert np.max(np.abs(lse[b, h][rows.numpy()] - ref_lse[rows].numpy())) < 1e-12
+
+
+def pin_bias_invariants(o):
+    """A constant M = c changes nothing but LSE, which moves by c; an M of
+    -inf above the diagonal is the causal mask; a scalar brute force."""
+    rng = _rng(51)
+    q = _rand(rng, 1, 1, 20, 4)
+    k = _rand(rng, 1, 1, 20, 4)
+    v = _rand(rng, 1, 1, 20, 4)
+    o1, l1 = o.attention_forward(q, k, v, False, 0.5)
+    o2, l2 = o.attention_forward(q, k, v, False, 0.5, bias=np.full((1, 1, 20, 20), 1.25))
+    assert np.max(np.abs(o1 - o2)) < 1e-12 and np.max(np.abs(l2 - l1 - 1.25)) < 1e-12
+    upper = np.where(np.triu(np.ones((20, 20)), 1) > 0, -np.inf, 0.0)[None, None]
+    o3, l3 = o.attention_forward(q, k, v, False, 0.5, bias=upper)
+    o4, l4 = o.attention_forward(q, k, v, True, 0.5)
+    assert np.max(np.abs(o3 - o4)) < 1e-12 and np.max(np.abs(l3 - l4)) < 1e-12
+    m = rng.standard_normal((1, 1, 20, 20))
+    out, lse = o.attention_forward(q, k, v, True, 0.5, bias=m)
+    for i in (0, 7, 19):
+        w = [math.exp(0.5 * math.fsum(q[0, 0, i, c] * k[0, 0, j, c] for c in range(4)) + m[0, 0, i, j])
+             for j in range(i + 1)]
+        z = math.fsum(w)
+        for c in range(4):
+            assert abs(out[0, 0, i, c] - math.fsum(wj * v[0, 0, j, c] for j, wj in enumerate(w)) / z) < 1e-12
+        assert abs(lse[0, 0, i] - math.log(z)) < 1e-12
+
+
 ALL_PINS = [
     pin_rows_sum_to_one,
     pin_constant_v,
@@ -557,4 +612,6 @@ ALL_PINS = [
     pin_fp8_attention,
     pin_block_mask_sdpa,
     pin_block_mask_brute,
+    pin_bias_sdpa,
+    pin_bias_invariants,
 ]

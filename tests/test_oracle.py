@@ -77,12 +77,12 @@ def _fresh_oracle():
 
 def _mut_drop_scale(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
-        q, k, 1.0, causal, row_offset, window_left, keep)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None: orig(
+        q, k, 1.0, causal, row_offset, window_left, keep, bias)
 
 
 def _mut_mask_includes_diagonal(m):
-    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
         s = float(scale) * (np.asarray(q, float) @ np.asarray(k, float).T)
         if causal:
             rows = np.arange(row_offset, row_offset + s.shape[0])[:, None]
@@ -93,7 +93,7 @@ def _mut_mask_includes_diagonal(m):
 
 
 def _mut_mask_off_by_one_late(m):
-    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
         s = float(scale) * (np.asarray(q, float) @ np.asarray(k, float).T)
         if causal:
             rows = np.arange(row_offset, row_offset + s.shape[0])[:, None]
@@ -105,12 +105,12 @@ def _mut_mask_off_by_one_late(m):
 
 def _mut_no_mask(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
-        q, k, scale, False, row_offset, window_left, keep)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None: orig(
+        q, k, scale, False, row_offset, window_left, keep, bias)
 
 
 def _mut_transposed_scores(m):
-    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
         q = np.asarray(q, float)
         k = np.asarray(k, float)
         s = float(scale) * (k @ q.T)
@@ -148,8 +148,8 @@ def _mut_softmax_wrong_axis(m):
 
 
 def _mut_pv_transposed(m):
-    def head(q, k, v, scale, causal, row_offset=0, window_left=None, keep=None):
-        s = m.attention_scores(q, k, scale, causal, row_offset, window_left, keep)
+    def head(q, k, v, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
+        s = m.attention_scores(q, k, scale, causal, row_offset, window_left, keep, bias)
         p, lse = m.softmax_with_lse(s)
         v = np.asarray(v, float)
         if p.shape[0] == p.shape[1]:
@@ -176,22 +176,22 @@ def _mut_page_no_table(m):
 
 def _mut_scale_squared(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
-        q, k, scale * scale, causal, row_offset, window_left, keep)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None: orig(
+        q, k, scale * scale, causal, row_offset, window_left, keep, bias)
 
 
 def _mut_window_off_by_one(m):
     orig = m.attention_scores
-    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None):
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
         w = None if window_left is None or window_left < 0 else window_left + 1
-        return orig(q, k, scale, causal, row_offset, w, keep)
+        return orig(q, k, scale, causal, row_offset, w, keep, bias)
     m.attention_scores = scores
 
 
 def _mut_window_ignored(m):
     orig = m.attention_scores
-    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None: orig(
-        q, k, scale, causal, row_offset, None, keep)
+    m.attention_scores = lambda q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None: orig(
+        q, k, scale, causal, row_offset, None, keep, bias)
 
 
 def _mut_append_shifted(m):
@@ -217,8 +217,8 @@ def _mut_append_ignores_table(m):
 
 def _mut_prefill_no_offset(m):
     orig = m.attention_head
-    def head(q, k, v, scale, causal, row_offset=0, window_left=None, keep=None):
-        return orig(q, k, v, scale, causal, 0, window_left, keep)
+    def head(q, k, v, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
+        return orig(q, k, v, scale, causal, 0, window_left, keep, bias)
     m.attention_head = head
 
 
@@ -278,6 +278,24 @@ def _mut_empty_rows_nan(m):
     m.softmax_with_lse = f
 
 
+def _mut_bias_before_scale(m):
+    orig = m.attention_scores
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
+        if bias is None:
+            return orig(q, k, scale, causal, row_offset, window_left, keep, None)
+        return orig(q, k, scale, causal, row_offset, window_left, keep, np.asarray(bias) * scale)
+    m.attention_scores = scores
+
+
+def _mut_bias_transposed(m):
+    orig = m.attention_scores
+    def scores(q, k, scale, causal, row_offset=0, window_left=None, keep=None, bias=None):
+        b = None if bias is None else (np.asarray(bias).T if np.asarray(bias).shape[0] == np.asarray(bias).shape[1]
+                                       else np.asarray(bias)[:, ::-1])
+        return orig(q, k, scale, causal, row_offset, window_left, keep, b)
+    m.attention_scores = scores
+
+
 MUTANTS = [
     _mut_drop_scale,
     _mut_scale_squared,
@@ -303,6 +321,8 @@ MUTANTS = [
     _mut_block_mask_transposed,
     _mut_block_mask_ignored,
     _mut_empty_rows_nan,
+    _mut_bias_before_scale,
+    _mut_bias_transposed,
 ]
 
 
