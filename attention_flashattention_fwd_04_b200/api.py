@@ -55,6 +55,8 @@ SIGNATURES = {
     "attn_device_status": (_c_i, [_c_p, ctypes.POINTER(ctypes.c_uint)]),
     "attn_fwd_block_sparse": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p,
                                      ctypes.c_longlong, ctypes.c_longlong, _c_p]),
+    "attn_fwd_bias": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_p,
+                             ctypes.c_longlong, ctypes.c_longlong, ctypes.c_longlong, _c_p]),
     "attn_fwd_fp8": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i, _c_f, _c_f, _c_f, _c_f,
                             _c_p]),
     "paged_kv_append": (_c_i, [_c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_p, _c_i, _c_i, _c_i, _c_i, _c_i, _c_i,
@@ -484,4 +486,45 @@ def attn_fwd_block_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kee
                                      Hkv, N, d, int(bool(causal)), float(scale), words.data_ptr(), b_stride, h_stride,
                                      _stream_handle(stream))
     _check(rc, "attn_fwd_block_sparse")
+    return out, lse
+
+
+def attn_fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: torch.Tensor, causal: bool = False,
+                  scale: float | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                  stream=None):
+    """attn_fwd with an additive mask M: softmax(scale * q k^T + M) v.
+
+    ``bias`` is bf16 [B or 1, Hq or 1, N or 1, N] (natural-log units, -inf
+    allowed), a strided view whose last dimension is contiguous and whose
+    other strides are multiples of 8 elements: e.g. a slice ``[..., :N]`` of a
+    buffer whose rows are padded to a multiple of 8.  Size-1 dimensions
+    broadcast (stride 0 is passed).  Rows whose scores are all -inf give
+    O = 0, LSE = -inf."""
+    _require(q, "q", torch.bfloat16, 4)
+    _require(k, "k", torch.bfloat16, 4)
+    _require(v, "v", torch.bfloat16, 4)
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} do not match q {tuple(q.shape)}")
+    if bias.dtype != torch.bfloat16 or bias.device != q.device or bias.dim() != 4:
+        raise ValueError("bias must be a 4-d bf16 tensor on q's device")
+    if (bias.shape[0] not in (1, B) or bias.shape[1] not in (1, Hq) or bias.shape[2] not in (1, N)
+            or bias.shape[3] != N):
+        raise ValueError(f"bias must be [1 or {B}, 1 or {Hq}, 1 or {N}, {N}], got {tuple(bias.shape)}")
+    if N > 1 and bias.stride(3) != 1:
+        raise ValueError("bias rows must be contiguous")
+    strides = [0 if bias.shape[i] == 1 else bias.stride(i) for i in range(3)]
+    if scale is None:
+        scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    _require(out, "out", torch.bfloat16, 4)
+    _require(lse, "lse", torch.float32, 3)
+    rc = lib().attn_fwd_bias(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, Hq, Hkv, N,
+                             d, int(bool(causal)), float(scale), bias.data_ptr(), strides[0], strides[1], strides[2],
+                             _stream_handle(stream))
+    _check(rc, "attn_fwd_bias")
     return out, lse

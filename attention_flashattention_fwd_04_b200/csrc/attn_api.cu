@@ -94,12 +94,14 @@ int sm_count() {
   return counts[dev];
 }
 
-template <int D, bool CAUSAL, bool WINDOW, bool PAGED = false, bool FP8 = false, bool SPARSE = false>
+template <int D, bool CAUSAL, bool WINDOW, bool PAGED = false, bool FP8 = false, bool SPARSE = false,
+          bool BIAS = false>
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const attn::PrefillParams& p, cudaStream_t stream) {
   using L = attn::PrefillLayout<D, PAGED, FP8, SPARSE>;
-  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED, FP8, SPARSE>;
-  cudaError_t e = ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED, FP8, SPARSE>>(L::kAlloc);
+  auto kernel = attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED, FP8, SPARSE, BIAS>;
+  cudaError_t e =
+      ensure_smem_limit<attn::prefill_fwd_kernel<D, CAUSAL, WINDOW, PAGED, FP8, SPARSE, BIAS>>(L::kAlloc);
   if (e != cudaSuccess) return fail_cuda(e);
   const int sms = sm_count();
   if (sms <= 0) return fail_cuda(cudaErrorInvalidDevice);
@@ -758,6 +760,68 @@ int attn_fwd_block_sparse(const attn_bf16* q, const attn_bf16* k, const attn_bf1
                   : launch_prefill<128, false, false, false, false, true>(tq, tk, tv, p, s);
   return causal ? launch_prefill<64, true, false, false, false, true>(tq, tk, tv, p, s)
                 : launch_prefill<64, false, false, false, false, true>(tq, tk, tv, p, s);
+}
+
+}  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Additive M
+// ----------------------------------------------------------------------------
+
+extern "C" {
+
+int attn_fwd_bias(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B,
+                  int Hq, int Hkv, int N, int d, int causal, float scale, const attn_bf16* bias,
+                  long long bias_b_stride, long long bias_h_stride, long long bias_row_stride, void* stream) {
+  if (!q || !k || !v || !o || !lse || !bias) return ATTN_ERR_NULL;
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return ATTN_ERR_SHAPE;
+  if (d != 64 && d != 128) return ATTN_ERR_SHAPE;
+  if (Hq % Hkv != 0) return ATTN_ERR_SHAPE;
+  if (causal != 0 && causal != 1) return ATTN_ERR_SHAPE;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return ATTN_ERR_SHAPE;
+  if (bias_b_stride < 0 || bias_h_stride < 0 || bias_row_stride < 0) return ATTN_ERR_SHAPE;
+  const long long padded = (static_cast<long long>(N) + 7) / 8 * 8;
+  if (bias_row_stride != 0 && bias_row_stride < padded) return ATTN_ERR_SHAPE;  // rows hold N (padded) values
+  const long long bh = static_cast<long long>(B) * Hq;
+  const long long blocks = (static_cast<long long>(N) + 255) / 256;
+  if (bh > INT_MAX || blocks * bh > INT_MAX) return ATTN_ERR_SHAPE;
+  if (misaligned16(q) || misaligned16(k) || misaligned16(v) || misaligned16(o) || misaligned16(bias) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u) != 0 || bias_b_stride % 8 != 0 || bias_h_stride % 8 != 0 ||
+      bias_row_stride % 8 != 0)
+    return ATTN_ERR_ALIGN;
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t row_bytes = static_cast<uint64_t>(d) * 2;
+  const uint64_t head_bytes = row_bytes * static_cast<uint64_t>(N);
+  if (!encode_3d(&tq, q, d, N, static_cast<uint64_t>(B) * Hq, row_bytes, head_bytes, 64, 128, 1) ||
+      !encode_3d(&tk, k, d, N, static_cast<uint64_t>(B) * Hkv, row_bytes, head_bytes, 64, 128, 1) ||
+      !encode_3d(&tv, v, d, N, static_cast<uint64_t>(B) * Hkv, row_bytes, head_bytes, 64, 128, 1))
+    return fail_cuda(cudaErrorInvalidValue);
+
+  attn::PrefillParams p{};
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.num_m = static_cast<int>(blocks);
+  p.num_items = static_cast<int>(blocks * bh);
+  p.window_left = -1;
+  p.scale_log2 = scale * kLog2e;
+  p.scale = scale;
+  p.o_scale = 1.f;
+  p.bias = reinterpret_cast<const __nv_bfloat16*>(bias);
+  p.bias_b_stride = bias_b_stride;
+  p.bias_h_stride = bias_h_stride;
+  p.bias_row_stride = bias_row_stride;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 128)
+    return causal ? launch_prefill<128, true, false, false, false, false, true>(tq, tk, tv, p, s)
+                  : launch_prefill<128, false, false, false, false, false, true>(tq, tk, tv, p, s);
+  return causal ? launch_prefill<64, true, false, false, false, false, true>(tq, tk, tv, p, s)
+                : launch_prefill<64, false, false, false, false, false, true>(tq, tk, tv, p, s);
 }
 
 }  // extern "C"

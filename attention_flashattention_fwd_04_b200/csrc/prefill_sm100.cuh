@@ -75,6 +75,7 @@ struct PrefillParams {
   int num_items;     // B * Hq * num_m (paged: counted on the device)
   int window_left;   // query i sees keys >= i - window_left (kernels with WINDOW only)
   float scale_log2;  // scale * log2(e) (FP8: times the Q and K descales)
+  float scale;       // the softmax scale itself (additive M only)
   float o_scale;     // FP8: the V descale, applied to O in the epilogue
   // Paged prefill (kernels with PAGED only): the new queries of sequence s
   // are packed rows cu_q[s] .. cu_q[s+1]-1; the cache holds seq_lens[s]
@@ -92,6 +93,11 @@ struct PrefillParams {
   const uint64_t* block_mask;
   long long mask_b_stride, mask_h_stride;
   int mask_words;              // ceil(ceil(N / 128) / 64), at most kMaskWords
+  // Additive M (kernels with BIAS only): bf16, natural-log units, row i of
+  // head (b, h) at bias + b * bias_b_stride + h * bias_h_stride + i * bias_row_stride
+  // (elements; rows padded to a multiple of 8, 16-byte aligned).
+  const __nv_bfloat16* bias;
+  long long bias_b_stride, bias_h_stride, bias_row_stride;
 };
 
 constexpr int kMaskWords = 4;  // block-sparse masks cover N <= 4 * 64 * 128 = 32768
@@ -447,7 +453,7 @@ __device__ __forceinline__ void reg_alloc_control() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 80;\n" ::: "memory");
 }
 
-template <int D, bool CAUSAL, bool WINDOW, bool PAGED, bool FP8 = false, bool SPARSE = false>
+template <int D, bool CAUSAL, bool WINDOW, bool PAGED, bool FP8 = false, bool SPARSE = false, bool BIAS = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -456,6 +462,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   static_assert(!(PAGED && WINDOW), "the paged kernels have no window");
   static_assert(!(FP8 && (PAGED || WINDOW)), "the FP8 kernels are dense, without a window");
   static_assert(!(SPARSE && (PAGED || WINDOW || FP8)), "the block-sparse kernels are dense bf16");
+  static_assert(!(BIAS && (PAGED || WINDOW || FP8 || SPARSE)), "the additive-M kernels are dense bf16");
   using L = PrefillLayout<D, PAGED, FP8, SPARSE>;
   constexpr int NS = L::NS;
   extern __shared__ uint8_t smem_raw[];
@@ -964,7 +971,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_arrive(bar(L::kBarStatsEmpty + 2 * t + slot));
         ++st_cnt[t];
         const int grow = it.m * 256 + t * 128 + row;  // query row of the head (paged: of the sequence's chunk)
-        const float inv_l = (FP8 ? p.o_scale : 1.f) / l_sum;  // FP8: l carries P's 2^8 as O does
+        // FP8: l carries P's 2^8 as O does.  Additive M can leave a row with
+        // no finite score (l = 0): O = 0, LSE = -inf.
+        const float inv_l = (BIAS && l_sum == 0.f) ? 0.f : (FP8 ? p.o_scale : 1.f) / l_sum;
         // O row / LSE index: dense [B, Hq, N, D] / [B, Hq, N]; paged by token, [total_q, Hq, D] / [total_q, Hq].
         const bool valid = grow < (PAGED ? it.n_q : p.N);
         const size_t row_index = PAGED ? (static_cast<size_t>(it.q0) + grow) * p.Hq + it.h
@@ -986,7 +995,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             dst[3] = make_uint4(w[12], w[13], w[14], w[15]);
           }
         }
-        if (valid) p.lse[row_index] = (m_used + log2f(l_sum) - (FP8 ? kFp8PLog2 : 0.f)) * kLn2;
+        if (valid)
+          p.lse[row_index] = (BIAS && l_sum == 0.f) ? -INFINITY
+                                                    : (m_used + log2f(l_sum) - (FP8 ? kFp8PLog2 : 0.f)) * kLn2;
         tc_fence_before();
         mbar_arrive(bar(L::kBarOFree + t));
       }
@@ -1029,15 +1040,50 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int j_set = lo_t - 1;  // block-sparse: the previous tile of this query tile's set
       for (int jj = 0; SPARSE ? next_bit_s(mw, j_set) < 64 * kMaskWords : jj < n_t; ++jj) {
         const int j = SPARSE ? (j_set = next_bit_s(mw, j_set)) : lo_t + jj;
+        const int kv0 = j * 128;
+        // Additive M: this row's 128 values of the tile, loaded (bf16, 16-byte
+        // vectors) while the MMA computes S.  Vectors past N and rows past N
+        // read nothing.
+        uint4 mb[BIAS ? 16 : 1];
+        if constexpr (BIAS) {
+          const __nv_bfloat16* brow = p.bias + it.b * p.bias_b_stride + it.h * p.bias_h_stride +
+                                      static_cast<long long>(grow) * p.bias_row_stride + kv0;
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            mb[v] = make_uint4(0u, 0u, 0u, 0u);
+            if (grow < p.N && kv0 + 8 * v < p.N) mb[v] = __ldg(reinterpret_cast<const uint4*>(brow) + v);
+          }
+        }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarSFull + t), s_cnt++ & 1u, kErrWaitSFull));
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld_x128_wait(s_addr, sr);
         float s[128];
+        if constexpr (BIAS) {
+          // s <- s * scale + M, in natural-log units; the exponent below turns
+          // them into log2 units (sl2_eff = log2(e)).  S comes out of tensor
+          // memory a quarter at a time, so each quarter's M registers die as
+          // it lands.
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-        const int kv0 = j * 128;
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t sr[32];
+            tmem_ld_x32_wait(s_addr + static_cast<uint32_t>(32 * q4), sr);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const uint32_t wv[4] = {mb[4 * q4 + v].x, mb[4 * q4 + v].y, mb[4 * q4 + v].z, mb[4 * q4 + v].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int c = 32 * q4 + 8 * v + 2 * i;
+                s[c] = fmaf(__uint_as_float(sr[c - 32 * q4]), p.scale, __uint_as_float(wv[i] << 16));
+                s[c + 1] = fmaf(__uint_as_float(sr[c + 1 - 32 * q4]), p.scale, __uint_as_float(wv[i] & 0xffff0000u));
+              }
+            }
+          }
+        } else {
+          uint32_t sr[128];
+          tmem_ld_x128_wait(s_addr, sr);
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        }
         // Tiles crossing the causal diagonal, a window's left edge or N get a
         // per-element mask (a select, so NaN-free -inf).
         if ((CAUSAL && kv0 + 127 > row0) || kv0 + 128 > n_kv ||
@@ -1070,7 +1116,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mx2 = fmaxf(mx2, s[126]);
         mx3 = fmaxf(mx3, s[127]);
         float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-        m_tile *= sl2;
+        const float sl2_eff = BIAS ? 1.4426950408889634f : sl2;  // additive M: scores in natural-log units
+        m_tile *= sl2_eff;
         const float m_new = fmaxf(m_used, m_tile);
         const bool upd = m_new > m_used + (FP8 ? kRescaleThresholdFp8 : kRescaleThreshold);
         const float alpha = upd ? ex2_approx(m_used - m_new) : 1.f;  // 0 on the first tile
@@ -1078,7 +1125,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         l_sum *= alpha;
         // FP8: P = 2^8 * 2^(s - m), the 2^8 folded into the offset.
         const float neg_m = (m_used == -INFINITY) ? 0.f : (FP8 ? kFp8PLog2 - m_used : -m_used);
-        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        const uint64_t sl2x2 = f2_pack(sl2_eff, sl2_eff);
         const uint64_t negm2 = f2_pack(neg_m, neg_m);
         // P in two halves, columns [0, 64) then [64, 128); each half goes to
         // tensor memory as soon as it is packed (fewer live registers).

@@ -243,6 +243,37 @@ def make_prefill_inputs(cfg: PrefillConfig, device: str | torch.device = "cpu"):
     return out
 
 
+def make_bias_inputs(shape, kind: str = "normal", seed: int = 0, sigma: float = 1.0, neg_inf_frac: float = 0.0,
+                     pad_fill: float = 0.0, device: str | torch.device = "cpu"):
+    """An additive mask M of ``shape`` = (B', H', R, N) (R = N, or 1 for one
+    row per head), bf16, natural-log units, as a view ``[..., :N]`` of a buffer
+    whose rows are padded to a multiple of 8 with ``pad_fill``.
+
+    kind "normal": N(0, sigma^2) values; kind "alibi": -slope_h * |i - j| with
+    slopes 2^(-8 (h + 1) / H') per head (a linear distance penalty).  A
+    fraction ``neg_inf_frac`` of the entries is then set to -inf.  Returns
+    (buffer, view)."""
+    Bp, Hp, R, N = shape
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    if kind == "normal":
+        m = torch.randn(Bp, Hp, R, N, generator=g, dtype=torch.float32) * sigma
+    elif kind == "alibi":
+        slopes = torch.pow(2.0, -8.0 * torch.arange(1, Hp + 1, dtype=torch.float32) / Hp)
+        i = torch.arange(R, dtype=torch.float32).view(R, 1)
+        j = torch.arange(N, dtype=torch.float32).view(1, N)
+        m = (-slopes.view(Hp, 1, 1) * (i - j).abs()).expand(Bp, Hp, R, N).clone()
+    else:
+        raise ValueError(kind)
+    if neg_inf_frac > 0:
+        m[torch.rand(m.shape, generator=g) < neg_inf_frac] = float("-inf")
+    padded = -(-N // 8) * 8
+    buf = torch.full((Bp, Hp, R, padded), pad_fill, dtype=torch.bfloat16)
+    buf[..., :N] = m.to(torch.bfloat16)
+    buf = buf.to(device)
+    return buf, buf[..., :N]
+
+
 def make_prefill_inputs_fp8(cfg: PrefillConfig, device: str | torch.device = "cpu"):
     """The bf16 draw of ``cfg`` quantised to e4m3 per tensor: descale =
     amax / 448, codes = round-to-nearest-even(x / descale) (PyTorch's

@@ -118,6 +118,28 @@ int attn_fwd_block_sparse(const attn_bf16* q, const attn_bf16* k, const attn_bf1
                           long long mask_b_stride, long long mask_h_stride, void* stream);
 
 /*
+ * attn_fwd_bias -- attn_fwd with a general additive mask M:
+ * softmax(scale * Q K^T + M) V ("FlashAttention-Style Kernels", the attention
+ * equation with M), M any finite values or -inf, added on top of the causal
+ * mask when causal = 1.
+ *   bias: bf16, natural-log units (the units of scale * q.k); M[i][j] of head
+ *     (b, h) at bias + b * bias_b_stride + h * bias_h_stride
+ *     + i * bias_row_stride + j (strides in elements, each >= 0 and a multiple
+ *     of 8; 0 broadcasts, e.g. bias_row_stride = 0 for one key-padding row per
+ *     head; bias 16-byte aligned).  Each row holds N values followed by
+ *     padding up to a multiple of 8 elements (read, then ignored: any bits),
+ *     so bias_row_stride, when not 0, is at least that padded length.
+ *     Read-only; owned by the caller.
+ * A query row whose scores are all -inf gets O = 0 and LSE = -inf.  +inf or
+ * NaN in M gives undefined (but in-bounds) results.  Other arguments and
+ * errors as attn_fwd; ATTN_ERR_SHAPE for negative or short strides,
+ * ATTN_ERR_ALIGN for strides that are not multiples of 8.
+ */
+int attn_fwd_bias(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, attn_bf16* o, float* lse, int B,
+                  int Hq, int Hkv, int N, int d, int causal, float scale, const attn_bf16* bias,
+                  long long bias_b_stride, long long bias_h_stride, long long bias_row_stride, void* stream);
+
+/*
  * attn_fwd_fp8 -- attn_fwd with e4m3 inputs (OCP FP8 E4M3 codes, one byte
  * each, same [B, H, N, d] layouts): the attention of q * q_descale,
  * k * k_descale and v * v_descale, the FP8 tensor-core path of FlashAttention

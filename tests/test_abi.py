@@ -204,3 +204,19 @@ def _bs(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=300, 
 ])
 def test_attn_fwd_block_sparse_rejects(lib, kw, code):
     assert _bs(lib, **kw) == code
+
+
+def _bias(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=300, d=128, causal=0, scale=0.1,
+          bias=FAKE, bs=0, hs=0, rs=304):
+    return lib.attn_fwd_bias(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, bias, bs, hs, rs, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bias=None), 1), (dict(o=None), 1),
+    (dict(N=0), 2), (dict(d=96), 2), (dict(Hq=3), 2), (dict(causal=2), 2), (dict(scale=float("nan")), 2),
+    (dict(bs=-8), 2), (dict(hs=-8), 2), (dict(rs=-8), 2), (dict(rs=296), 2), (dict(rs=300), 2),
+    (dict(bias=FAKE + 8), 3), (dict(q=FAKE + 4), 3), (dict(bs=12), 3), (dict(hs=4), 3), (dict(rs=305), 3),
+    (dict(lse=FAKE + 2), 3),
+])
+def test_attn_fwd_bias_rejects(lib, kw, code):
+    assert _bias(lib, **kw) == code

@@ -112,3 +112,15 @@ def test_window_flops():
     N, Wl = lw.N, lw.window_left
     pairs = (Wl + 1) * (Wl + 2) // 2 + (N - Wl - 1) * (Wl + 1)  # ramp, then full windows
     assert W.prefill_flops(lw) == 4.0 * lw.B * lw.Hq * lw.d * pairs
+
+
+def test_bias_inputs_layout_and_values():
+    buf, view = W.make_bias_inputs((1, 4, 5, 13), "alibi", pad_fill=float("nan"))
+    assert buf.shape == (1, 4, 5, 16) and view.shape == (1, 4, 5, 13)
+    assert view.stride(2) == 16 and view.stride(3) == 1
+    assert torch.isnan(buf[..., 13:]).all()
+    # head 0 of 4: slope 2^-2; entry (i, j) = -|i - j| / 4
+    assert float(view[0, 0, 4, 1]) == -0.75 and float(view[0, 0, 2, 2]) == 0.0
+    _, v2 = W.make_bias_inputs((2, 1, 3, 20), "normal", seed=3, neg_inf_frac=0.5)
+    frac = torch.isneginf(v2.float()).float().mean().item()
+    assert 0.2 < frac < 0.8
