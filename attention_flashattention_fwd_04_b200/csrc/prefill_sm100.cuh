@@ -133,13 +133,12 @@ struct PrefillLayout {
   // [kPagedMaxBlocks], cu_q [S+1], seq_lens [S], the block count and 16 ints
   // of scan scratch.
   // Block-sparse: the current item's KV-tile sets, as words in shared memory
-  // (read back on use, so the loops hold none in registers): the MMA
-  // thread's both sets, the producer's union, one query tile's set per
-  // softmax warp.
+  // (read back on use, so the loops hold none in registers): the producer's
+  // union and one query tile's set per softmax warp; then the item's tiles as
+  // the MMA warp lists them (16-bit entries, up to 256).
   static constexpr int kSeq = kStats + kStatsBytes;
-  // The MMA thread also lists the item's tiles (16-bit entries, up to 256).
-  static constexpr int kMaskMma = 0, kMaskProd = 8, kMaskSoftmax = 12;  // in words, from kSeq
-  static constexpr int kTileList = (8 + 4 + 8 * 4) * 8;                  // bytes, from kSeq
+  static constexpr int kMaskProd = 0, kMaskSoftmax = 4;  // in words, from kSeq
+  static constexpr int kTileList = (4 + 8 * 4) * 8;      // bytes, from kSeq
   static constexpr int kSeqBytes = PAGED ? (kPagedMaxBlocks + 2 * kPagedMaxSeqs + 1 + 1 + 16) * 4
                                          : SPARSE ? kTileList + 64 * kMaskWords * 2 : 0;
   static constexpr int kBar = (kSeq + kSeqBytes + 7) / 8 * 8;
@@ -703,8 +702,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           mbar_wait(bar(L::kBarVFull + j % NS), static_cast<uint32_t>(j / NS) & 1u, kErrWaitDrain);
       }
       __syncwarp();
-    } else if (warp == 13 && lane == 0) {
+    } else if (warp == 13 && (SPARSE || lane == 0)) {
       // ---------------------------------------------------------- MMA issuer
+      // (lane 0; block-sparse: the whole warp lists each item's tiles)
       constexpr uint32_t idesc_qk =
           FP8 ? make_idesc_e4m3(128, 128, false, false) : make_idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = FP8 ? make_idesc_e4m3(128, D, false, true) : make_idesc_bf16(128, D, false, true);
@@ -724,11 +724,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int kk = 0; kk < kSSteps; ++kk) {
           const uint32_t off = static_cast<uint32_t>((kk >> 2) * L::kBoxBytes + (kk & 3) * 32);
           if constexpr (FP8)
-            mma_f8_ss(d_tmem, make_sdesc_sw128(q_addr + off, 16, 1024), make_sdesc_sw128(k_addr + off, 16, 1024),
-                      idesc_qk, kk > 0 ? 1u : 0u);
+            mma_f8_ss_lo(d_tmem, sdesc_sw128_lo<16>(q_addr + off), sdesc_sw128_lo<16>(k_addr + off), idesc_qk,
+                         kk > 0 ? 1u : 0u);
           else
-            mma_bf16_ss(d_tmem, make_sdesc_sw128(q_addr + off, 16, 1024),
-                        make_sdesc_sw128(k_addr + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+            mma_bf16_ss_lo(d_tmem, sdesc_sw128_lo<16>(q_addr + off), sdesc_sw128_lo<16>(k_addr + off), idesc_qk,
+                           kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(L::kBarSFull + t));
       };
@@ -739,11 +739,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kPvSteps; ++kk) {
           // P: 32 bytes of a row per step = 8 TMEM columns; V: kPvKeys rows of 128 bytes.
-          const uint64_t vdesc = make_sdesc_sw128(v_addr + kk * kPvKeys * 128, L::kBoxBytes, 1024);
+          const uint32_t vdesc = sdesc_sw128_lo<L::kBoxBytes>(v_addr + kk * kPvKeys * 128);
           if constexpr (FP8)
-            mma_f8_ts(o_tmem, p_tmem + kk * 8, vdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+            mma_f8_ts_lo(o_tmem, p_tmem + kk * 8, vdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
           else
-            mma_bf16_ts(o_tmem, p_tmem + kk * 8, vdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
+            mma_bf16_ts_lo(o_tmem, p_tmem + kk * 8, vdesc, idesc_pv, (accumulate || kk > 0) ? 1u : 0u);
         }
       };
       PrefillItem it;
@@ -752,35 +752,52 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // the item walks their union.
         uint32_t q_cnt = 0;  // items whose Q was loaded (every item except fully masked block-sparse ones)
         for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
-          // This thread's copy of the item's two sets (shared memory, re-read on use).
-          volatile uint64_t* const mm0 = mask_smem + L::kMaskMma;
-          volatile uint64_t* const mm1 = mm0 + kMaskWords;
-#pragma unroll
-          for (int k = 0; k < kMaskWords; ++k) {
-            mm0[k] = it.mk0[k];
-            mm1[k] = it.mk1[k];
-          }
           // The item's tiles in order, one 16-bit entry each: tile index (bits
           // 0-7), visited by query tile 0 / 1 (bits 8, 9), first for it
-          // (10, 11), last for it (12, 13).  Listed while Q is in flight.
+          // (10, 11), last for it (12, 13).  Listed by the whole warp while Q
+          // is in flight: lane l takes tiles 8l .. 8l+7 of the item's mask
+          // words (already limited to the tiles each query tile can see) and
+          // writes them at the prefix sum of the lower lanes' counts.
           volatile uint16_t* const tl = reinterpret_cast<volatile uint16_t*>(smem + L::kSeq + L::kTileList);
-          int n_u = 0;
+          int n_u;
           {
-            int seen0 = 0, seen1 = 0;
-            for (int j = next_bit_union_s(mm0, mm1, it.jb - 1); j < it.je; j = next_bit_union_s(mm0, mm1, j)) {
-              const int a = bit_s(mm0, j), b = bit_s(mm1, j);
-              int e = j | (a << 8) | (b << 9);
-              if (a && !seen0) e |= 1 << 10;
-              if (b && !seen1) e |= 1 << 11;
-              if (a && next_bit_s(mm0, j) >= 64 * kMaskWords) e |= 1 << 12;
-              if (b && next_bit_s(mm1, j) >= 64 * kMaskWords) e |= 1 << 13;
-              seen0 |= a;
-              seen1 |= b;
-              tl[n_u++] = static_cast<uint16_t>(e);
+            static_assert(kMaskWords == 4, "one mask word per 8 lanes");
+            const int kw = lane >> 3;
+            const uint64_t w0 = kw == 0 ? it.mk0[0] : kw == 1 ? it.mk0[1] : kw == 2 ? it.mk0[2] : it.mk0[3];
+            const uint64_t w1 = kw == 0 ? it.mk1[0] : kw == 1 ? it.mk1[1] : kw == 2 ? it.mk1[2] : it.mk1[3];
+            const int sh = (lane & 7) * 8;
+            const uint32_t b0 = static_cast<uint32_t>(w0 >> sh) & 0xffu;
+            const uint32_t b1 = static_cast<uint32_t>(w1 >> sh) & 0xffu;
+            const uint32_t ub = b0 | b1;
+            int incl = __popc(ub);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const int y = __shfl_up_sync(0xffffffffu, incl, o);
+              if (lane >= o) incl += y;
             }
+            n_u = __shfl_sync(0xffffffffu, incl, 31);
+            const uint32_t any0 = __ballot_sync(0xffffffffu, b0 != 0u);
+            const uint32_t any1 = __ballot_sync(0xffffffffu, b1 != 0u);
+            // This lane's bit (if any) that is the first / last tile of set 0 / 1.
+            const int f0 = (lane == __ffs(any0) - 1) ? __ffs(b0) - 1 : -1;
+            const int f1 = (lane == __ffs(any1) - 1) ? __ffs(b1) - 1 : -1;
+            const int l0 = (any0 != 0u && lane == 31 - __clz(any0)) ? 31 - __clz(b0) : -1;
+            const int l1 = (any1 != 0u && lane == 31 - __clz(any1)) ? 31 - __clz(b1) : -1;
+            int pos = incl - __popc(ub);
+            for (uint32_t rest = ub; rest != 0u; rest &= rest - 1u) {
+              const int b = __ffs(rest) - 1;
+              int e = (8 * lane + b) | static_cast<int>(((b0 >> b) & 1u) << 8) | static_cast<int>(((b1 >> b) & 1u) << 9);
+              if (b == f0) e |= 1 << 10;
+              if (b == f1) e |= 1 << 11;
+              if (b == l0) e |= 1 << 12;
+              if (b == l1) e |= 1 << 13;
+              tl[pos++] = static_cast<uint16_t>(e);
+            }
+            __syncwarp();
           }
           if (n_u == 0) continue;  // nothing to compute (the epilogue writes zeros)
           auto on = [&](int t, int e) { return ((e >> (8 + t)) & 1) != 0; };
+          if (lane == 0) do {  // the item's MMAs; break = give up (ok false)
           if (!(ok = mbar_wait(bar(L::kBarQFull), q_cnt & 1u, kErrWaitQ))) break;
           ++q_cnt;
           {
@@ -855,6 +872,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           if (!ok) break;
           kv_it += u;
+          } while (false);
+          // The list is rewritten only after lane 0 is done with it.
+          ok = __shfl_sync(0xffffffffu, ok, 0);
         }
       } else {
         // Dense: query tile t visits the contiguous range [lo(t), hi(t)).
@@ -926,8 +946,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       // All issued MMAs must finish before tensor memory is released.
-      mma_commit(bar(L::kBarMmaDone));
-      mbar_wait(bar(L::kBarMmaDone), 0, kErrWaitMmaDone);
+      if (lane == 0) {
+        mma_commit(bar(L::kBarMmaDone));
+        mbar_wait(bar(L::kBarMmaDone), 0, kErrWaitMmaDone);
+      }
     }
     __syncwarp();
   } else if (wg == 2) {
