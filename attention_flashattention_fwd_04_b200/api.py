@@ -458,8 +458,11 @@ def attn_fwd_block_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kee
                           causal: bool = True, scale: float | None = None, out: torch.Tensor | None = None,
                           lse: torch.Tensor | None = None, stream=None):
     """attn_fwd with a block-sparse mask: ``keep`` boolean [B or 1, Hq or 1,
-    ceil(N/128), ceil(N/128)] (1 = the 128x128 block is computed).  Rows
-    that see no key give O = 0, LSE = -inf."""
+    ceil(N/128), ceil(N/128)] (1 = the 128x128 block is computed), or the
+    same mask already packed by ``pack_block_mask`` (int64 words [B or 1,
+    Hq or 1, ceil(N/128), ceil(ceil(N/128)/64)], on q's device; a caller
+    that reuses one mask packs it once).  Rows that see no key give O = 0,
+    LSE = -inf."""
     _require(q, "q", torch.bfloat16, 4)
     _require(k, "k", torch.bfloat16, 4)
     _require(v, "v", torch.bfloat16, 4)
@@ -468,10 +471,18 @@ def attn_fwd_block_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kee
     if k.shape != (B, Hkv, N, d) or v.shape != k.shape:
         raise ValueError(f"k/v shape {tuple(k.shape)}/{tuple(v.shape)} do not match q {tuple(q.shape)}")
     nb = -(-N // 128)
-    if keep.dim() != 4 or keep.shape[2:] != (nb, nb) or keep.shape[0] not in (1, B) or keep.shape[1] not in (1, Hq):
-        raise ValueError(f"keep must be [1 or {B}, 1 or {Hq}, {nb}, {nb}], got {tuple(keep.shape)}")
-    words = pack_block_mask(keep.to(q.device)).contiguous()
-    nw = words.shape[-1]
+    nw = -(-nb // 64)
+    if keep.dtype == torch.int64:
+        if (keep.dim() != 4 or keep.shape[2:] != (nb, nw) or keep.shape[0] not in (1, B)
+                or keep.shape[1] not in (1, Hq) or keep.device != q.device or not keep.is_contiguous()):
+            raise ValueError(f"packed mask must be contiguous int64 [1 or {B}, 1 or {Hq}, {nb}, {nw}] on q's "
+                             f"device, got {tuple(keep.shape)}")
+        words = keep
+    else:
+        if (keep.dim() != 4 or keep.shape[2:] != (nb, nb) or keep.shape[0] not in (1, B)
+                or keep.shape[1] not in (1, Hq)):
+            raise ValueError(f"keep must be [1 or {B}, 1 or {Hq}, {nb}, {nb}], got {tuple(keep.shape)}")
+        words = pack_block_mask(keep.to(q.device)).contiguous()
     h_stride = 0 if keep.shape[1] == 1 else nb * nw
     b_stride = 0 if keep.shape[0] == 1 else keep.shape[1] * nb * nw
     if scale is None:

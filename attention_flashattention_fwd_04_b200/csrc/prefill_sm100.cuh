@@ -134,13 +134,16 @@ struct PrefillLayout {
   // of scan scratch.
   // Block-sparse: the current item's KV-tile sets, as words in shared memory
   // (read back on use, so the loops hold none in registers): the producer's
-  // union and one query tile's set per softmax warp; then the item's tiles as
-  // the MMA warp lists them (16-bit entries, up to 256).
+  // union and one query tile's set per softmax warp; then two tile lists
+  // (16-bit entries, up to 256 each) and their lengths, written by the lister
+  // warp one item ahead of the MMA thread.
   static constexpr int kSeq = kStats + kStatsBytes;
   static constexpr int kMaskProd = 0, kMaskSoftmax = 4;  // in words, from kSeq
   static constexpr int kTileList = (4 + 8 * 4) * 8;      // bytes, from kSeq
+  static constexpr int kTileListBytes = 64 * kMaskWords * 2;
+  static constexpr int kTileCount = kTileList + 2 * kTileListBytes;  // two ints
   static constexpr int kSeqBytes = PAGED ? (kPagedMaxBlocks + 2 * kPagedMaxSeqs + 1 + 1 + 16) * 4
-                                         : SPARSE ? kTileList + 64 * kMaskWords * 2 : 0;
+                                         : SPARSE ? kTileCount + 2 * 4 : 0;
   static constexpr int kBar = (kSeq + kSeqBytes + 7) / 8 * 8;
   static constexpr int kBarQFull = 0;
   static constexpr int kBarQEmpty = 1;
@@ -155,7 +158,9 @@ struct PrefillLayout {
   static constexpr int kBarStatsFull = kBarOFree + 2;   // [tile][slot]
   static constexpr int kBarStatsEmpty = kBarStatsFull + 4;
   static constexpr int kBarMmaDone = kBarStatsEmpty + 4;
-  static constexpr int kNumBars = kBarMmaDone + 1;
+  static constexpr int kBarListFull = kBarMmaDone + 1;    // 2: block-sparse tile lists
+  static constexpr int kBarListEmpty = kBarListFull + 2;  // 2
+  static constexpr int kNumBars = kBarListEmpty + 2;
   static constexpr int kTmemSlot = kBar + kNumBars * 8;
   static constexpr int kBytes = kTmemSlot + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack: the base is rounded up to 1024 B
@@ -509,6 +514,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar(L::kBarStatsEmpty + i), 128);
     }
     mbar_init(bar(L::kBarMmaDone), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::kBarListFull + i), 1);
+      mbar_init(bar(L::kBarListEmpty + i), 1);
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -702,9 +711,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           mbar_wait(bar(L::kBarVFull + j % NS), static_cast<uint32_t>(j / NS) & 1u, kErrWaitDrain);
       }
       __syncwarp();
-    } else if (warp == 13 && (SPARSE || lane == 0)) {
+    } else if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      // (lane 0; block-sparse: the whole warp lists each item's tiles)
       constexpr uint32_t idesc_qk =
           FP8 ? make_idesc_e4m3(128, 128, false, false) : make_idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = FP8 ? make_idesc_e4m3(128, D, false, true) : make_idesc_bf16(128, D, false, true);
@@ -751,53 +759,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // Block-sparse: each query tile visits an arbitrary set of KV tiles;
         // the item walks their union.
         uint32_t q_cnt = 0;  // items whose Q was loaded (every item except fully masked block-sparse ones)
-        for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
-          // The item's tiles in order, one 16-bit entry each: tile index (bits
-          // 0-7), visited by query tile 0 / 1 (bits 8, 9), first for it
-          // (10, 11), last for it (12, 13).  Listed by the whole warp while Q
-          // is in flight: lane l takes tiles 8l .. 8l+7 of the item's mask
-          // words (already limited to the tiles each query tile can see) and
-          // writes them at the prefix sum of the lower lanes' counts.
-          volatile uint16_t* const tl = reinterpret_cast<volatile uint16_t*>(smem + L::kSeq + L::kTileList);
-          int n_u;
-          {
-            static_assert(kMaskWords == 4, "one mask word per 8 lanes");
-            const int kw = lane >> 3;
-            const uint64_t w0 = kw == 0 ? it.mk0[0] : kw == 1 ? it.mk0[1] : kw == 2 ? it.mk0[2] : it.mk0[3];
-            const uint64_t w1 = kw == 0 ? it.mk1[0] : kw == 1 ? it.mk1[1] : kw == 2 ? it.mk1[2] : it.mk1[3];
-            const int sh = (lane & 7) * 8;
-            const uint32_t b0 = static_cast<uint32_t>(w0 >> sh) & 0xffu;
-            const uint32_t b1 = static_cast<uint32_t>(w1 >> sh) & 0xffu;
-            const uint32_t ub = b0 | b1;
-            int incl = __popc(ub);
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const int y = __shfl_up_sync(0xffffffffu, incl, o);
-              if (lane >= o) incl += y;
-            }
-            n_u = __shfl_sync(0xffffffffu, incl, 31);
-            const uint32_t any0 = __ballot_sync(0xffffffffu, b0 != 0u);
-            const uint32_t any1 = __ballot_sync(0xffffffffu, b1 != 0u);
-            // This lane's bit (if any) that is the first / last tile of set 0 / 1.
-            const int f0 = (lane == __ffs(any0) - 1) ? __ffs(b0) - 1 : -1;
-            const int f1 = (lane == __ffs(any1) - 1) ? __ffs(b1) - 1 : -1;
-            const int l0 = (any0 != 0u && lane == 31 - __clz(any0)) ? 31 - __clz(b0) : -1;
-            const int l1 = (any1 != 0u && lane == 31 - __clz(any1)) ? 31 - __clz(b1) : -1;
-            int pos = incl - __popc(ub);
-            for (uint32_t rest = ub; rest != 0u; rest &= rest - 1u) {
-              const int b = __ffs(rest) - 1;
-              int e = (8 * lane + b) | static_cast<int>(((b0 >> b) & 1u) << 8) | static_cast<int>(((b1 >> b) & 1u) << 9);
-              if (b == f0) e |= 1 << 10;
-              if (b == f1) e |= 1 << 11;
-              if (b == l0) e |= 1 << 12;
-              if (b == l1) e |= 1 << 13;
-              tl[pos++] = static_cast<uint16_t>(e);
-            }
-            __syncwarp();
+        for (int r = 0; ok; ++r) {
+          // The item's tile list, from the lister warp (length -1: no items left).
+          const int buf = r & 1;
+          if (!(ok = mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>(r >> 1) & 1u, kErrWaitList))) break;
+          const volatile uint16_t* const tl =
+              reinterpret_cast<const volatile uint16_t*>(smem + L::kSeq + L::kTileList + buf * L::kTileListBytes);
+          const int n_u = reinterpret_cast<const volatile int*>(smem + L::kSeq + L::kTileCount)[buf];
+          if (n_u < 0) break;
+          if (n_u == 0) {  // nothing to compute (the epilogue writes zeros)
+            mbar_arrive(bar(L::kBarListEmpty + buf));
+            continue;
           }
-          if (n_u == 0) continue;  // nothing to compute (the epilogue writes zeros)
           auto on = [&](int t, int e) { return ((e >> (8 + t)) & 1) != 0; };
-          if (lane == 0) do {  // the item's MMAs; break = give up (ok false)
           if (!(ok = mbar_wait(bar(L::kBarQFull), q_cnt & 1u, kErrWaitQ))) break;
           ++q_cnt;
           {
@@ -872,9 +846,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           if (!ok) break;
           kv_it += u;
-          } while (false);
-          // The list is rewritten only after lane 0 is done with it.
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          mbar_arrive(bar(L::kBarListEmpty + buf));  // the list may be rewritten
         }
       } else {
         // Dense: query tile t visits the contiguous range [lo(t), hi(t)).
@@ -946,9 +918,68 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       // All issued MMAs must finish before tensor memory is released.
-      if (lane == 0) {
-        mma_commit(bar(L::kBarMmaDone));
-        mbar_wait(bar(L::kBarMmaDone), 0, kErrWaitMmaDone);
+      mma_commit(bar(L::kBarMmaDone));
+      mbar_wait(bar(L::kBarMmaDone), 0, kErrWaitMmaDone);
+    } else if (SPARSE && warp == 14) {
+      // ---------------------------------------------------------- tile lister
+      // Block-sparse: lists each item's tiles in order, one item ahead of the
+      // MMA thread, one 16-bit entry per tile: tile index (bits 0-7), visited
+      // by query tile 0 / 1 (bits 8, 9), first for it (10, 11), last for it
+      // (12, 13).  Lane l takes tiles 8l .. 8l+7 of the item's mask words
+      // (already limited to the tiles each query tile can see) and writes them
+      // at the prefix sum of the lower lanes' counts.
+      PrefillItem it;
+      for (int r = 0;; ++r) {
+        const bool have = prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq);
+        const int buf = r & 1;
+        if (r >= 2) {  // the MMA thread is done with the list of item r - 2
+          int okw = 1;
+          if (lane == 0)
+            okw = mbar_wait(bar(L::kBarListEmpty + buf), static_cast<uint32_t>((r >> 1) - 1) & 1u, kErrWaitList);
+          if (__shfl_sync(0xffffffffu, okw, 0) == 0) break;
+        }
+        volatile uint16_t* const tl =
+            reinterpret_cast<volatile uint16_t*>(smem + L::kSeq + L::kTileList + buf * L::kTileListBytes);
+        int n_u = -1;
+        if (have) {
+          static_assert(kMaskWords == 4, "one mask word per 8 lanes");
+          const int kw = lane >> 3;
+          const uint64_t w0 = kw == 0 ? it.mk0[0] : kw == 1 ? it.mk0[1] : kw == 2 ? it.mk0[2] : it.mk0[3];
+          const uint64_t w1 = kw == 0 ? it.mk1[0] : kw == 1 ? it.mk1[1] : kw == 2 ? it.mk1[2] : it.mk1[3];
+          const int sh = (lane & 7) * 8;
+          const uint32_t b0 = static_cast<uint32_t>(w0 >> sh) & 0xffu;
+          const uint32_t b1 = static_cast<uint32_t>(w1 >> sh) & 0xffu;
+          const uint32_t ub = b0 | b1;
+          int incl = __popc(ub);
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          n_u = __shfl_sync(0xffffffffu, incl, 31);
+          const uint32_t any0 = __ballot_sync(0xffffffffu, b0 != 0u);
+          const uint32_t any1 = __ballot_sync(0xffffffffu, b1 != 0u);
+          // This lane's bit (if any) that is the first / last tile of set 0 / 1.
+          const int f0 = (lane == __ffs(any0) - 1) ? __ffs(b0) - 1 : -1;
+          const int f1 = (lane == __ffs(any1) - 1) ? __ffs(b1) - 1 : -1;
+          const int l0 = (any0 != 0u && lane == 31 - __clz(any0)) ? 31 - __clz(b0) : -1;
+          const int l1 = (any1 != 0u && lane == 31 - __clz(any1)) ? 31 - __clz(b1) : -1;
+          int pos = incl - __popc(ub);
+          for (uint32_t rest = ub; rest != 0u; rest &= rest - 1u) {
+            const int b = __ffs(rest) - 1;
+            int e = (8 * lane + b) | static_cast<int>(((b0 >> b) & 1u) << 8) | static_cast<int>(((b1 >> b) & 1u) << 9);
+            if (b == f0) e |= 1 << 10;
+            if (b == f1) e |= 1 << 11;
+            if (b == l0) e |= 1 << 12;
+            if (b == l1) e |= 1 << 13;
+            tl[pos++] = static_cast<uint16_t>(e);
+          }
+        }
+        if (lane == 0) reinterpret_cast<volatile int*>(smem + L::kSeq + L::kTileCount)[buf] = n_u;
+        __threadfence_block();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::kBarListFull + buf));  // release: the entries above are visible
+        if (!have) break;
       }
     }
     __syncwarp();

@@ -33,6 +33,7 @@ enum : unsigned int {
   kErrDecodeWait = 1u << 10,
   kErrDecodeTable = 1u << 11,
   kErrPagedTable = 1u << 12,  // paged prefill / append: a length or block-table entry out of range
+  kErrWaitList = 1u << 13,    // block-sparse prefill: the tile-list handoff
 };
 
 // Wall-clock limit for one wait (ns).  Real waits in these kernels last

@@ -254,24 +254,67 @@ def make_bias_inputs(shape, kind: str = "normal", seed: int = 0, sigma: float = 
     fraction ``neg_inf_frac`` of the entries is then set to -inf.  Returns
     (buffer, view)."""
     Bp, Hp, R, N = shape
+    padded = -(-N // 8) * 8
+    buf = torch.full((Bp, Hp, R, padded), pad_fill, dtype=torch.bfloat16)
     g = torch.Generator(device="cpu")
     g.manual_seed(seed)
     if kind == "normal":
-        m = torch.randn(Bp, Hp, R, N, generator=g, dtype=torch.float32) * sigma
+        buf[..., :N] = (torch.randn(Bp, Hp, R, N, generator=g, dtype=torch.float32) * sigma).to(torch.bfloat16)
     elif kind == "alibi":
-        slopes = torch.pow(2.0, -8.0 * torch.arange(1, Hp + 1, dtype=torch.float32) / Hp)
-        i = torch.arange(R, dtype=torch.float32).view(R, 1)
-        j = torch.arange(N, dtype=torch.float32).view(1, N)
-        m = (-slopes.view(Hp, 1, 1) * (i - j).abs()).expand(Bp, Hp, R, N).clone()
+        for h in range(Hp):  # one head at a time: no full-size float32 intermediate
+            buf[:, h, :, :N] = alibi_rows(Hp, h, 0, R, N)
     else:
         raise ValueError(kind)
     if neg_inf_frac > 0:
-        m[torch.rand(m.shape, generator=g) < neg_inf_frac] = float("-inf")
-    padded = -(-N // 8) * 8
-    buf = torch.full((Bp, Hp, R, padded), pad_fill, dtype=torch.bfloat16)
-    buf[..., :N] = m.to(torch.bfloat16)
+        view = buf[..., :N]
+        view[torch.rand(view.shape, generator=g) < neg_inf_frac] = float("-inf")
     buf = buf.to(device)
     return buf, buf[..., :N]
+
+
+def alibi_rows(Hp: int, h: int, r0: int, r1: int, N: int) -> torch.Tensor:
+    """Rows r0 .. r1-1 of head h's linear distance penalty (of Hp heads):
+    -s_h * |i - j| with s_h = 2^(-8 (h + 1) / Hp), bf16 [r1 - r0, N]."""
+    s = 2.0 ** (-8.0 * (h + 1) / Hp)
+    i = torch.arange(r0, r1, dtype=torch.float32).view(-1, 1)
+    j = torch.arange(N, dtype=torch.float32).view(1, -1)
+    return (-s * (i - j).abs()).to(torch.bfloat16)
+
+
+def longformer_keep(nb: int) -> torch.Tensor:
+    """Block mask [nb, nb] (128 x 128 blocks) of a Longformer-style pattern:
+    each query block keeps its own key block, the one before it, and key
+    block 0 (a global first block)."""
+    keep = torch.zeros(nb, nb, dtype=torch.bool)
+    for i in range(nb):
+        keep[i, max(0, i - 1): i + 1] = True
+        keep[i, 0] = True
+    return keep
+
+
+def block_sparse_pairs(keep2d, N: int, causal: bool) -> int:
+    """Visible (query, key) pairs of one head under a [nb, nb] block mask of
+    128 x 128 blocks (and the causal mask)."""
+    import numpy as np
+    keep2d = np.asarray(keep2d, dtype=bool)
+    nb = keep2d.shape[0]
+    total = 0
+    for qb in range(nb):
+        rows = np.arange(qb * 128, min(N, qb * 128 + 128))
+        for kb in np.nonzero(keep2d[qb])[0]:
+            c0, c1 = kb * 128, min(N, kb * 128 + 128)
+            if causal:
+                total += int(np.clip(np.minimum(rows + 1, c1) - c0, 0, None).sum())
+            else:
+                total += rows.size * (c1 - c0)
+    return total
+
+
+# Prefill workloads with a general mask: (shapes, mask kind).
+MASK_WORKLOADS = {
+    "longformer_sparse": ("causal_gqa", "longformer"),
+    "alibi_bias": ("causal_gqa", "alibi"),
+}
 
 
 def make_prefill_inputs_fp8(cfg: PrefillConfig, device: str | torch.device = "cpu"):

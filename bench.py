@@ -174,6 +174,36 @@ PREFILL_WORKLOADS = ("default", "causal_mha", "causal_gqa", "long_causal", "long
 DECODE_WORKLOADS = ("default", "paged_decode", "small_decode")
 CHUNKED_WORKLOADS = ("chunked_prefill",)
 FP8_WORKLOADS = {"causal_gqa_fp8": "causal_gqa", "long_causal_fp8": "long_causal"}  # e4m3 inputs, same shapes
+MASK_WORKLOADS = W.MASK_WORKLOADS  # block-sparse / additive-M prefill on the same shapes
+
+
+def mask_label(kind: str) -> str:
+    return {"longformer": "block-sparse Longformer mask (diagonal + previous + first 128-blocks)",
+            "alibi": "additive M per head, -2^(-8(h+1)/H)|i-j| (bf16)"}[kind]
+
+
+def mask_inputs(kind: str, c):
+    """Host-side mask of a mask workload: the block keep matrix [1, 1, nb, nb]
+    or the per-head M buffer (rows padded to a multiple of 8) and its view."""
+    if kind == "longformer":
+        from attention_flashattention_fwd_04_b200.api import pack_block_mask
+        nb = -(-c.N // 128)
+        return {"keep": pack_block_mask(W.longformer_keep(nb).view(1, 1, nb, nb))}  # int64 words, packed once
+    buf, _ = W.make_bias_inputs((1, c.Hq, c.N, c.N), "alibi")
+    return {"bias_buf": buf}
+
+
+def mask_work(kind: str, c):
+    """(FLOPs, bytes that the same kernel moves while it computes): visible
+    pairs x 4d; for M also its visible values (2 B each, every head its own)
+    plus Q, K, V, O and LSE, which then bound the kernel as much as the
+    tensor cores do."""
+    if kind == "longformer":
+        pairs = W.block_sparse_pairs(W.longformer_keep(-(-c.N // 128)), c.N, c.causal)
+        return 4.0 * c.d * pairs * c.B * c.Hq, 0.0
+    pairs = c.N * (c.N + 1) // 2 if c.causal else c.N * c.N
+    qkvo = 2.0 * c.B * c.N * c.d * (2 * c.Hq + 2 * c.Hkv) + 4.0 * c.B * c.Hq * c.N
+    return 4.0 * c.d * pairs * c.B * c.Hq, 2.0 * pairs * c.B * c.Hq + qkvo
 
 
 def chunked_label(c) -> str:
@@ -181,10 +211,12 @@ def chunked_label(c) -> str:
             f"context {c.ctx_range[0]}..{c.ctx_range[1]} new {c.q_range[0]}..{c.q_range[1]}")
 
 
-def prefill_label(c, fp8=False) -> str:
+def prefill_label(c, fp8=False, mask_kind=None) -> str:
     mask = ("fp8 " if fp8 else "") + ("causal" if c.causal else "full")
     if c.window_left >= 0:
         mask += f" window={c.window_left}"
+    if mask_kind is not None:
+        mask += " + " + mask_label(mask_kind)
     return f"{mask} prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}"
 
 class Step:
@@ -202,8 +234,11 @@ class Step:
             base = W.CHUNKED_CONFIGS[workload]
             self.chunked_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
         self.fp8 = workload in FP8_WORKLOADS
-        if workload in PREFILL_WORKLOADS or self.fp8:
-            name = "causal_mha" if workload == "default" else FP8_WORKLOADS.get(workload, workload)
+        self.mask_kind = MASK_WORKLOADS[workload][1] if workload in MASK_WORKLOADS else None
+        self.fused_bytes = 0.0  # bytes moved by the prefill kernel itself while it computes
+        if workload in PREFILL_WORKLOADS or self.fp8 or self.mask_kind is not None:
+            name = ("causal_mha" if workload == "default" else
+                    FP8_WORKLOADS.get(workload, MASK_WORKLOADS.get(workload, (workload,))[0]))
             base = W.PREFILL_CONFIGS[name]
             self.prefill_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
         if workload in DECODE_WORKLOADS:
@@ -222,6 +257,9 @@ class Step:
                 q, k, v = W.make_prefill_inputs(c)
             self.host.update(q=q, k=k, v=v)
             self.flops = W.prefill_flops(c)
+            if self.mask_kind is not None:
+                self.host.update(mask_inputs(self.mask_kind, c))
+                self.flops, self.fused_bytes = mask_work(self.mask_kind, c)
         if self.decode_cfg is not None:
             c = self.decode_cfg
             inp = W.make_decode_inputs(c)
@@ -298,6 +336,14 @@ class Step:
             qd, kd, vd = self.descales
             self.api.attn_fwd_fp8(d["q"], d["k"], d["v"], c.causal, c.scale, qd, kd, vd, out=d["o"], lse=d["lse"])
             return
+        if self.mask_kind == "longformer":
+            self.api.attn_fwd_block_sparse(d["q"], d["k"], d["v"], d["keep"], c.causal, c.scale, out=d["o"],
+                                           lse=d["lse"])
+            return
+        if self.mask_kind == "alibi":
+            self.api.attn_fwd_bias(d["q"], d["k"], d["v"], d["bias_buf"][..., :c.N], c.causal, c.scale, out=d["o"],
+                                   lse=d["lse"])
+            return
         self.api.attn_fwd(d["q"], d["k"], d["v"], c.causal, c.scale, out=d["o"], lse=d["lse"],
                           window_left=c.window_left if c.window_left >= 0 else None)
 
@@ -317,7 +363,11 @@ class Step:
         return peaks["bf16_tflops"] * (2.0 if self.fp8 else 1.0)
 
     def ideal_seconds(self, peaks) -> float:
-        return self.flops / (self.tensor_peak_tflops(peaks) * 1e12) + self.bytes / (peaks["hbm_gbs"] * 1e9)
+        """Separate kernels add up; within the prefill kernel the tensor work
+        and the bytes it moves overlap, so the slower of the two counts."""
+        prefill = max(self.flops / (self.tensor_peak_tflops(peaks) * 1e12),
+                      self.fused_bytes / (peaks["hbm_gbs"] * 1e9))
+        return prefill + self.bytes / (peaks["hbm_gbs"] * 1e9)
 
 
 def config_dict(step: Step, n_gpus: int):
@@ -325,11 +375,15 @@ def config_dict(step: Step, n_gpus: int):
     parts = []
     if step.prefill_cfg is not None:
         c = step.prefill_cfg
-        parts.append(prefill_label(c, step.fp8))
+        parts.append(prefill_label(c, step.fp8, step.mask_kind))
         cfg["prefill"] = {"B": c.B, "Hq": c.Hq, "Hkv": c.Hkv, "N": c.N, "d": c.d, "causal": c.causal,
                           "window_left": c.window_left, "scale": c.scale, "seed": c.seed,
                           "value_scale": c.value_scale, "k_offset_sigma": c.k_offset_sigma, "flops": step.flops,
                           "inputs": "e4m3, per-tensor descale amax/448" if step.fp8 else "bf16"}
+        if step.mask_kind is not None:
+            cfg["prefill"]["mask"] = mask_label(step.mask_kind)
+            if step.fused_bytes:
+                cfg["prefill"]["bytes"] = step.fused_bytes
     if step.chunked_cfg is not None:
         c, inp = step.chunked_cfg, step.chunked_inp
         parts.append(chunked_label(c))
@@ -368,7 +422,7 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
 
     import oracle
 
-    prefill_cfg, decode_cfg, host, decode_inp, chunked, fp8 = step_cfgs
+    prefill_cfg, decode_cfg, host, decode_inp, chunked, fp8, mask = step_cfgs
     flops = 0.0
     nbytes = 0.0
     done_heads = 0
@@ -411,13 +465,22 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
                 hk = h * c.Hkv // c.Hq
                 r0 = c.N - rows
                 wl = c.window_left if c.window_left >= 0 else None
+                keep = bias = None
+                if mask is not None and mask[0] == "longformer":
+                    keep = oracle.block_keep(mask[1], np.arange(r0, c.N), c.N)
+                elif mask is not None:
+                    bias = mask[1](h, r0)  # rows r0..N-1 of head h's M
                 oracle.attention_head(q[b, h, r0:], k[b, hk], v[b, hk], c.scale, c.causal, row_offset=r0,
-                                      window_left=wl)
+                                      window_left=wl, keep=keep, bias=bias)
                 # visible (query, key) pairs of rows r0..N-1
                 i = np.arange(r0, c.N)
-                last = i if c.causal else np.full_like(i, c.N - 1)
-                first = np.maximum(i - wl, 0) if wl is not None else np.zeros_like(i)
-                flops += 4.0 * float(np.sum(last - first + 1)) * c.d
+                if keep is not None:
+                    vis = keep & (np.arange(c.N)[None, :] <= i[:, None]) if c.causal else keep
+                    flops += 4.0 * float(vis.sum()) * c.d
+                else:
+                    last = i if c.causal else np.full_like(i, c.N - 1)
+                    first = np.maximum(i - wl, 0) if wl is not None else np.zeros_like(i)
+                    flops += 4.0 * float(np.sum(last - first + 1)) * c.d
                 done_heads += 1
                 if time.perf_counter() - t0 > budget_s / (2 if decode_cfg is not None else 1):
                     break
@@ -441,13 +504,24 @@ def oracle_sample(step_cfgs, budget_s: float, per_call=False):
     seconds = time.perf_counter() - t0
     desc = []
     if prefill_cfg is not None:
-        desc.append(f"{done_heads} prefill heads ({'last 128 rows' if per_call else 'all rows'})")
+        desc.append(f"{done_heads} prefill heads ({'last 128 rows' if per_call else 'all rows'})"
+                    + (f" with the {mask_label(mask[0])}" if mask is not None else ""))
     if decode_cfg is not None:
         desc.append(f"{done_seqs} decode sequences")
     if chunked is not None:
         desc.append(f"append of all chunks + attention of {done_chunks} "
                     f"{'chunk tails (last 128 rows)' if per_call else 'whole chunks'}")
     return {"flops": flops, "bytes": nbytes}, seconds, ", ".join(desc)
+
+
+def oracle_mask(kind: str, c):
+    """The mask of a mask workload as the oracle takes it: the [nb, nb] block
+    matrix, or a function giving rows r0..N-1 of head h's M (built row-wise by
+    the same generator, so no full-size M is needed on the host)."""
+    import numpy as np
+    if kind == "longformer":
+        return kind, W.longformer_keep(-(-c.N // 128)).numpy()
+    return kind, lambda h, r0: W.alibi_rows(c.Hq, h, r0, c.N, c.N).float().numpy().astype(np.float64)
 
 
 def cpu_threads() -> int:
@@ -469,7 +543,7 @@ def run_reference(args, world, rank):
         return None
     peaks = load_peaks()
     step = StepHost(args.workload)
-    cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp, step.chunked, step.fp8)
+    cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp, step.chunked, step.fp8, step.mask)
     for _ in range(args.warmup):
         oracle_sample(cfgs, 0.0, per_call=True)
     work_f = work_b = secs = 0.0
@@ -481,6 +555,10 @@ def run_reference(args, world, rank):
         secs += s
     tpk = peaks["bf16_tflops"] * (2.0 if step.fp8 is not None else 1.0)  # e4m3: nominal 2x bf16
     ideal = work_f / (tpk * 1e12) + work_b / (peaks["hbm_gbs"] * 1e9)
+    if step.mask is not None and step.mask[0] == "alibi":
+        # the sampled rows' share of the kernel's bytes, overlapping its FLOPs as on the GPU
+        fl, by = mask_work("alibi", step.prefill_cfg)
+        ideal = max(ideal, work_f * by / fl / (peaks["hbm_gbs"] * 1e9))
     value = ideal / secs
     line = {
         "metric": METRIC, "value": value, "unit": unit_string(), "n_gpus": world, "steps": args.steps,
@@ -503,6 +581,7 @@ class StepHost:
         self.decode_inp = None
         self.chunked = None
         self.fp8 = None
+        self.mask = None
         parts = []
         if workload in FP8_WORKLOADS:
             self.prefill_cfg = W.PREFILL_CONFIGS[FP8_WORKLOADS[workload]]
@@ -519,6 +598,13 @@ class StepHost:
             q, k, v = W.make_prefill_inputs(self.prefill_cfg)
             self.host.update(q=q, k=k, v=v)
             parts.append(prefill_label(self.prefill_cfg))
+        if workload in MASK_WORKLOADS:
+            name, kind = MASK_WORKLOADS[workload]
+            c = self.prefill_cfg = W.PREFILL_CONFIGS[name]
+            q, k, v = W.make_prefill_inputs(c)
+            self.host.update(q=q, k=k, v=v)
+            self.mask = oracle_mask(kind, c)
+            parts.append(prefill_label(c, mask_kind=kind))
         if workload in DECODE_WORKLOADS:
             self.decode_cfg = W.DECODE_CONFIGS["small_decode" if workload == "small_decode" else "paged_decode"]
             inp = W.make_decode_inputs(self.decode_cfg)
@@ -631,6 +717,12 @@ def run_ours(args, world, rank, local_rank):
         kernels["prefill_fwd_kernel"] = {"bound": "tensor", "achieved": tfl, "peak": tpk,
                                          "unit": "TFLOP/s", "frac": tfl / tpk,
                                          "us_per_launch": per * 1e6, "algorithmic": step.flops}
+        if step.fused_bytes / (peaks["hbm_gbs"] * 1e9) > step.flops / (tpk * 1e12):
+            # the kernel's own bytes (a per-head M) take longer than its FLOPs: HBM is its roof
+            gbs = step.fused_bytes / per / 1e9
+            kernels["prefill_fwd_kernel"].update(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                                                 frac=gbs / peaks["hbm_gbs"], algorithmic=step.fused_bytes,
+                                                 tflops=tfl)
         line["prefill_tflops"] = tfl
     if step.decode_cfg is not None:
         per = t_decode / args.steps
@@ -655,13 +747,15 @@ def run_ours(args, world, rank, local_rank):
     dominant = max(kernels, key=lambda k: kernels[k]["us_per_launch"])
     traffic = load_traffic()
     dk = kernels[dominant]
+    # Records are keyed by the bench workload whose launches ncu captured; the
+    # default step's two kernels were captured in their own workloads.
     if dominant.startswith("prefill"):
-        cfg_name = (step.prefill_cfg or step.chunked_cfg).name
-        tr = traffic.get(("prefill_fwd_kernel", cfg_name))
+        tr = traffic.get(("prefill_fwd_kernel", "causal_mha" if args.workload == "default" else args.workload))
     elif dominant == "paged_append_kernel":
-        tr = traffic.get(("paged_append_kernel", step.chunked_cfg.name))
+        tr = traffic.get(("paged_append_kernel", args.workload))
     else:
-        parts = [traffic.get((k, step.decode_cfg.name)) for k in ("decode_split_kernel", "decode_merge_kernel")]
+        key = "paged_decode" if args.workload == "default" else args.workload
+        parts = [traffic.get((k, key)) for k in ("decode_split_kernel", "decode_merge_kernel")]
         tr = None if any(x is None for x in parts) else sum(parts)
     peak_source = f"{peaks['source']} (burst)"
     if step.fp8 and dominant.startswith("prefill"):
@@ -674,7 +768,9 @@ def run_ours(args, world, rank, local_rank):
         chunked = (step.chunked_cfg, step.chunked_inp) if step.chunked_cfg is not None else None
         w, secs, desc = oracle_sample((step.prefill_cfg, step.decode_cfg, step.host,
                                        getattr(step, "decode_inp", None), chunked,
-                                       step.descales if step.fp8 else None), args.cpu_seconds)
+                                       step.descales if step.fp8 else None,
+                                       oracle_mask(step.mask_kind, step.prefill_cfg) if step.mask_kind else None),
+                                      args.cpu_seconds)
         ideal = w["flops"] / (step.tensor_peak_tflops(peaks) * 1e12) + w["bytes"] / (peaks["hbm_gbs"] * 1e9)
         cpu = {"value": ideal / secs, "unit": unit_string(), "cores": cpu_threads(), "kind": "oracle",
                "sample": f"{desc}; {secs:.1f} s"}
@@ -737,7 +833,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="default",
                     choices=sorted(set(PREFILL_WORKLOADS) | set(DECODE_WORKLOADS) | set(CHUNKED_WORKLOADS) |
-                                   set(FP8_WORKLOADS)))
+                                   set(FP8_WORKLOADS) | set(MASK_WORKLOADS)))
     ap.add_argument("--decode-graph", action="store_true",
                     help="run the decode step as a captured CUDA graph (split pass + merge)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

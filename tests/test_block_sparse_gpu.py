@@ -99,3 +99,16 @@ def test_longformer_pattern_full_size_sampled():
         rows = [0, 127, 128, 255, 4000, 8191]
         ro, rl = oracle.attention_rows(qf, kf, vf, True, cfg.scale, 0, h, rows, block_mask=full)
         check(o[0, h, rows].numpy().astype(np.float64), lse[0, h, rows].numpy().astype(np.float64), ro, rl)
+
+
+def test_packed_mask_equals_boolean_mask():
+    """The binding takes the mask already packed (int64 words, packed once by
+    the caller) as well as boolean: the same words reach the kernel."""
+    cfg = W.PrefillConfig("t", 2, 4, 2, 900, 128, True, seed=73)
+    nb = -(-cfg.N // 128)
+    keep = torch.from_numpy(np.random.default_rng(5).random((2, 1, nb, nb)) < 0.5)
+    q, k, v = (t.cuda() for t in W.make_prefill_inputs(cfg))
+    o1, l1 = api.attn_fwd_block_sparse(q, k, v, keep.cuda(), True, cfg.scale)
+    o2, l2 = api.attn_fwd_block_sparse(q, k, v, api.pack_block_mask(keep).cuda(), True, cfg.scale)
+    assert api.device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
