@@ -106,6 +106,9 @@ PREFILL_CONFIGS = {
     "long_causal": PrefillConfig("long_causal", 1, 8, 8, 32768, 128, True, 5, k_offset_sigma=2.0),
     "long_window": PrefillConfig("long_window", 1, 8, 8, 32768, 128, True, 7, k_offset_sigma=2.0,
                                  window_left=4095),
+    # causal_gqa cut to 4 query heads (one KV head): a per-head M of 0.5 GB
+    # instead of 4.3 GB, small enough for a full ncu capture.
+    "causal_gqa_h4": PrefillConfig("causal_gqa_h4", 1, 4, 1, 8192, 128, True, 3, value_scale=0.5),
 }
 
 DECODE_CONFIGS = {
@@ -314,6 +317,7 @@ def block_sparse_pairs(keep2d, N: int, causal: bool) -> int:
 MASK_WORKLOADS = {
     "longformer_sparse": ("causal_gqa", "longformer"),
     "alibi_bias": ("causal_gqa", "alibi"),
+    "alibi_bias_h4": ("causal_gqa_h4", "alibi"),
 }
 
 
