@@ -203,7 +203,7 @@ def mask_work(kind: str, c):
         return 4.0 * c.d * pairs * c.B * c.Hq, 0.0
     pairs = c.N * (c.N + 1) // 2 if c.causal else c.N * c.N
     qkvo = 2.0 * c.B * c.N * c.d * (2 * c.Hq + 2 * c.Hkv) + 4.0 * c.B * c.Hq * c.N
-    return 4.0 * c.d * pairs * c.B * c.Hq, 2.0 * pairs * c.B * c.Hq + qkvo
+    return W.prefill_flops(c), 2.0 * pairs * c.B * c.Hq + qkvo  # FLOPs: the dense lines' N^2/2 convention
 
 
 def chunked_label(c) -> str:

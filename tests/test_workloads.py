@@ -124,3 +124,51 @@ def test_bias_inputs_layout_and_values():
     _, v2 = W.make_bias_inputs((2, 1, 3, 20), "normal", seed=3, neg_inf_frac=0.5)
     frac = torch.isneginf(v2.float()).float().mean().item()
     assert 0.2 < frac < 0.8
+
+
+def test_block_sparse_pairs_brute_force():
+    """Visible pairs under a block mask (and causality) against a count over
+    the expanded element mask."""
+    import numpy as np
+    rng = np.random.default_rng(3)
+    for N, causal in ((300, True), (300, False), (129, True), (1000, True)):
+        nb = -(-N // 128)
+        keep = rng.random((nb, nb)) < 0.5
+        elem = keep[np.arange(N)[:, None] // 128, np.arange(N)[None, :] // 128]
+        if causal:
+            elem &= np.arange(N)[None, :] <= np.arange(N)[:, None]
+        assert W.block_sparse_pairs(keep, N, causal) == int(elem.sum())
+    # all ones and causal: every pair with j <= i
+    assert W.block_sparse_pairs(np.ones((3, 3), bool), 300, True) == 300 * 301 // 2
+
+
+def test_longformer_keep_pattern():
+    keep = W.longformer_keep(5)
+    assert keep.dtype == torch.bool and keep.shape == (5, 5)
+    assert keep[:, 0].all()                                   # global first block
+    assert all(keep[i, i] and keep[i, i - 1] for i in range(1, 5))
+    assert int(keep.sum()) == 1 + 2 + 3 + 3 + 3               # row 0: {0}; row 1: {0,1}; rows 2+: {0,i-1,i}
+
+
+def test_alibi_rows_match_the_full_generator():
+    buf, view = W.make_bias_inputs((1, 3, 40, 37), "alibi")
+    for h in range(3):
+        assert torch.equal(W.alibi_rows(3, h, 5, 40, 37), view[0, h, 5:])
+
+
+def test_bench_mask_work_accounting():
+    """FLOPs and bytes bench.py credits the mask workloads with."""
+    import bench
+    c = W.PREFILL_CONFIGS["causal_gqa"]
+    f, b = bench.mask_work("longformer", c)
+    assert b == 0.0
+    assert f == 4.0 * c.d * W.block_sparse_pairs(W.longformer_keep(c.N // 128), c.N, True) * c.B * c.Hq
+    f, b = bench.mask_work("alibi", c)
+    pairs = c.N * (c.N + 1) // 2
+    assert f == W.prefill_flops(c) == 4.0 * c.d * c.N * c.N / 2 * c.Hq   # the dense lines' convention
+    m_bytes = 2.0 * pairs * c.Hq                                  # every head its own M
+    qkvo = 2.0 * c.N * c.d * (2 * c.Hq + 2 * c.Hkv) + 4.0 * c.Hq * c.N
+    assert b == m_bytes + qkvo
+    # the per-head M makes this prefill HBM-bound at the measured peaks
+    peaks = bench.load_peaks()
+    assert b / (peaks["hbm_gbs"] * 1e9) > f / (peaks["bf16_tflops"] * 1e12)
