@@ -345,23 +345,29 @@ __global__ void __launch_bounds__(256)
   const float* plse = p.part_lse + static_cast<size_t>(wid) * p.max_splits;
   const float* po = p.part_o + static_cast<size_t>(wid) * p.max_splits * D + lane * kPer;
   constexpr float kLog2e = 1.4426950408889634f;
-  float mx = -INFINITY;
-  for (int t = lane; t < n_splits; t += 32) mx = fmaxf(mx, plse[t]);
+  // The first 32 splits' LSEs stay in registers (lane t: split t) for the
+  // weights; the partial rows are then read 16 splits per round, so a
+  // sequence of up to 32 splits costs three dependent trips to memory.
+  const float pl0 = lane < n_splits ? plse[lane] : -INFINITY;
+  float mx = pl0;
+  for (int t = lane + 32; t < n_splits; t += 32) mx = fmaxf(mx, plse[t]);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
   float wsum = 0.f;
   float out[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) out[e] = 0.f;
+  constexpr int kRound = 16;  // splits whose rows are in flight at once
   for (int t0 = 0; t0 < n_splits; t0 += 32) {
     const int cnt = min(32, n_splits - t0);
-    const float my_w = lane < cnt ? ex2_approx((plse[t0 + lane] - mx) * kLog2e) : 0.f;
+    const float pl = t0 == 0 ? pl0 : (lane < cnt ? plse[t0 + lane] : -INFINITY);
+    const float my_w = lane < cnt ? ex2_approx((pl - mx) * kLog2e) : 0.f;
     wsum += my_w;
-    for (int i = 0; i < cnt; i += 8) {
-      float v[8][kPer];
-      float w[8];
+    for (int i = 0; i < cnt; i += kRound) {
+      float v[kRound][kPer];
+      float w[kRound];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < kRound; ++u) {
         w[u] = __shfl_sync(0xffffffffu, my_w, (i + u) & 31);
         if (i + u < cnt) {
           const float* src = po + static_cast<size_t>(t0 + i + u) * D;
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(256)
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
+      for (int u = 0; u < kRound; ++u)
 #pragma unroll
         for (int e = 0; e < kPer; ++e) out[e] = fmaf(w[u], v[u][e], out[e]);
     }

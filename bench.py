@@ -44,6 +44,14 @@ METRIC = "causal prefill TFLOP/s and paged-decode KV GB/s, as fraction of B200 p
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 KERNEL_SOURCES = ("attn_api.cu", "prefill_sm100.cuh", "decode_sm100.cuh", "paged_append.cuh", "ptx.cuh", "tmem_ldst.cuh",
                   "exp2_poly.cuh")
+# The sources each kernel is built from (the launch code in attn_api.cu included): an ncu
+# record stays valid while these are unchanged.
+KERNEL_SOURCE_SETS = {
+    "prefill_fwd_kernel": ("attn_api.cu", "prefill_sm100.cuh", "ptx.cuh", "tmem_ldst.cuh", "exp2_poly.cuh"),
+    "decode_split_kernel": ("attn_api.cu", "decode_sm100.cuh", "ptx.cuh"),
+    "decode_merge_kernel": ("attn_api.cu", "decode_sm100.cuh", "ptx.cuh"),
+    "paged_append_kernel": ("attn_api.cu", "paged_append.cuh", "ptx.cuh"),
+}
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -60,9 +68,10 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, bf16_tflops_sustained=FALLBACK_PEAKS["bf16_tflops"])
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str | None = None) -> str:
+    """Hash of one kernel's sources (all kernel sources when None)."""
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in (KERNEL_SOURCE_SETS[kernel] if kernel else KERNEL_SOURCES):
         with open(os.path.join(ROOT, "attention_flashattention_fwd_04_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -84,8 +93,7 @@ def load_traffic():
                     out[(kv["kernel"], kv.get("bench"))] = (kv.get("sha"), float(kv["dram_bytes_per_launch"]))
     except OSError:
         return {}
-    sha = kernel_source_hash()
-    return {k: v for k, (s, v) in out.items() if s == sha}
+    return {k: v for k, (s, v) in out.items() if k[0] in KERNEL_SOURCE_SETS and s == kernel_source_hash(k[0])}
 
 
 def shard_seed(base_seed: int, rank: int) -> int:

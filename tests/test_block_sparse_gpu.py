@@ -112,3 +112,27 @@ def test_packed_mask_equals_boolean_mask():
     o2, l2 = api.attn_fwd_block_sparse(q, k, v, api.pack_block_mask(keep).cuda(), True, cfg.scale)
     assert api.device_status() == 0
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("N,causal", [(32768, True), (20000, False)])
+def test_multi_word_masks_sampled(N, causal):
+    """More than 64 key blocks: the mask rows span several uint64 words (four
+    at N = 32768, the limit), so every lane of the tile lister and every word
+    of each set is used.  Sampled rows against the oracle."""
+    cfg = W.PrefillConfig("t", 1, 2, 1, N, 128, causal, seed=74)
+    nb = -(-N // 128)
+    rng = np.random.default_rng(N)
+    keep = rng.random((1, 2, nb, nb)) < 0.15
+    keep[0, 0, :, nb - 1] = True                   # the last key block (top bits of the last word)
+    keep[0, 1, :, 63:65] = True                    # blocks on both sides of the first word boundary
+    keep[0, 1, 100, :] = False                     # a query block that sees nothing
+    q, k, v = W.make_prefill_inputs(cfg)
+    o, lse = api.attn_fwd_block_sparse(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(keep).cuda(), causal,
+                                       cfg.scale)
+    assert api.device_status() == 0
+    o, lse = o.float().cpu(), lse.cpu()
+    rows = [0, 127, 128, 8191, 8192, 100 * 128 + 5, 16384, N - 129, N - 1]
+    for h in (0, 1):
+        ro, rl = oracle.attention_rows(q.float(), k.float(), v.float(), causal, cfg.scale, 0, h, rows,
+                                       block_mask=keep[0:1])
+        check(o[0, h, rows].numpy().astype(np.float64), lse[0, h, rows].numpy().astype(np.float64), ro, rl)
