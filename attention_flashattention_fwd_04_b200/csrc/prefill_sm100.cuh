@@ -145,9 +145,9 @@ struct PrefillLayout {
   static constexpr int kSeqBytes = PAGED ? (kPagedMaxBlocks + 2 * kPagedMaxSeqs + 1 + 1 + 16) * 4
                                          : SPARSE ? kTileCount + 2 * 4 : 0;
   static constexpr int kBar = (kSeq + kSeqBytes + 7) / 8 * 8;
-  static constexpr int kBarQFull = 0;
-  static constexpr int kBarQEmpty = 1;
-  static constexpr int kBarKFull = 2;
+  static constexpr int kBarQFull = 0;   // [tile]
+  static constexpr int kBarQEmpty = 2;  // [tile]
+  static constexpr int kBarKFull = 4;
   static constexpr int kBarKEmpty = kBarKFull + NS;
   static constexpr int kBarVFull = kBarKEmpty + NS;
   static constexpr int kBarVEmpty = kBarVFull + NS;
@@ -281,6 +281,39 @@ __device__ __forceinline__ bool paged_item(int idx, const PrefillParams& p, cons
   it.jb = 0;
   it.je = max(it.hi0, it.hi1);
   return true;
+}
+
+// The value, through a move the compiler cannot see into: what is derived
+// from it is computed where it is used rather than hoisted and kept live.
+__device__ __forceinline__ uint32_t opaque_u32(uint32_t x) {
+  uint32_t y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Non-blocking: has the phase with this parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "selp.u32 %0, 1, 0, p;\n"
+      "}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Whether this CTA has an item in round `round` (prefill_item without the item).
+template <bool PAGED>
+__device__ __forceinline__ bool prefill_item_exists(int round, const PrefillParams& p, const PagedSeqs& sq) {
+  const int G = static_cast<int>(gridDim.x);
+  const int c = static_cast<int>(blockIdx.x);
+  const int idx = round * G + ((round & 1) ? (G - 1 - c) : c);
+  if constexpr (PAGED) return idx / p.Hq < *sq.nblocks;
+  return idx < p.num_items;
 }
 
 template <bool CAUSAL, bool WINDOW, bool PAGED = false, bool SPARSE = false>
@@ -493,8 +526,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(L::kBarQFull), 1);
-    mbar_init(bar(L::kBarQEmpty), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::kBarQFull + t), 1);
+      mbar_init(bar(L::kBarQEmpty + t), 1);
+    }
     for (int s = 0; s < NS; ++s) {
       mbar_init(bar(L::kBarKFull + s), 1);
       mbar_init(bar(L::kBarKEmpty + s), 1);
@@ -538,7 +573,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // ---------------------------------------------------------- producer
       // Lane 0 waits and issues the copies; the paged kernels also use the
       // other lanes for block-table lookups and the partly used last page.
-      int kv_it = 0, k_issued = 0, v_issued = 0, q_issued = 0;
+      int kv_it = 0, k_issued = 0, v_issued = 0;
+      int q_issued[2] = {0, 0};  // loads of Q tile t
       bool ok = true;
       PrefillItem it{};
       // Paged: the tile whose pages t_row / t_valid describe (lane b: box b),
@@ -681,19 +717,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // The item's first K tile first: it can land while the previous item
         // still holds Q.
         if (!(ok = load_k(j0, kz))) break;
-        if (q_issued > 0 &&
-            !(ok = wait0(bar(L::kBarQEmpty), static_cast<uint32_t>(q_issued - 1) & 1u, kErrWaitQ)))
-          break;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar(L::kBarQFull), (it.has(1) ? 2 : 1) * L::kTileBytes);
-          for (int c = 0; c < L::kBoxes; ++c)
-            tma_load_3d(base + L::kQ0 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * L::kBoxCols, qrow, qz);
-          if (it.has(1))
+        // Q0 and Q1 are released separately, each after its query tile's last
+        // S of the previous item, so Q0 can arrive while Q1 is still in use.
+        for (int t = 0; t < 2; ++t) {
+          if (t == 1 && !it.has(1)) break;
+          if (q_issued[t] > 0 &&
+              !(ok = wait0(bar(L::kBarQEmpty + t), static_cast<uint32_t>(q_issued[t] - 1) & 1u, kErrWaitQ)))
+            break;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(bar(L::kBarQFull + t), L::kTileBytes);
             for (int c = 0; c < L::kBoxes; ++c)
-              tma_load_3d(base + L::kQ1 + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull), c * L::kBoxCols, qrow + 128,
-                          qz);
+              tma_load_3d(base + (t ? L::kQ1 : L::kQ0) + c * L::kBoxBytes, &tm_q, bar(L::kBarQFull + t),
+                          c * L::kBoxCols, qrow + 128 * t, qz);
+          }
+          ++q_issued[t];
         }
-        ++q_issued;
+        if (!ok) break;
         if (!(ok = load_v(j0, kz))) break;
         ++kv_it;
         for (int j = unext(j0); j < it.je; j = unext(j), ++kv_it) {
@@ -703,8 +742,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       // Every copy this warp started must land before the CTA may exit.
       if (lane == 0) {
-        if (q_issued > 0)
-          mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(q_issued - 1) & 1u, kErrWaitDrain);
+        for (int t = 0; t < 2; ++t)
+          if (q_issued[t] > 0)
+            mbar_wait(bar(L::kBarQFull + t), static_cast<uint32_t>(q_issued[t] - 1) & 1u, kErrWaitDrain);
         for (int j = max(0, k_issued - NS); j < k_issued; ++j)
           mbar_wait(bar(L::kBarKFull + j % NS), static_cast<uint32_t>(j / NS) & 1u, kErrWaitDrain);
         for (int j = max(0, v_issued - NS); j < v_issued; ++j)
@@ -716,6 +756,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t idesc_qk =
           FP8 ? make_idesc_e4m3(128, 128, false, false) : make_idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = FP8 ? make_idesc_e4m3(128, D, false, true) : make_idesc_bf16(128, D, false, true);
+      // The next item's first S0 is issued early in the FP8 kernel, whose
+      // shorter MMA leg leaves the tile-0 softmax waiting at item boundaries;
+      // in the bf16 kernels the extra issue work costs more than it saves.
+      constexpr bool kEarlyS0 = FP8;
       // Every MMA takes 32 bytes of its K dimension: 16 bf16 or 32 e4m3.
       constexpr int kSSteps = D * L::kElemBytes / 32;     // S = Q K^T over the head dim
       constexpr int kPvKeys = 32 / L::kElemBytes;         // keys per P V step
@@ -725,8 +769,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t o_cnt[2] = {0u, 0u};  // items whose O_t has been completed
       bool ok = true;
       auto issue_s = [&](int t, int st) {
-        const uint32_t q_addr = base + (t ? L::kQ1 : L::kQ0);
-        const uint32_t k_addr = base + L::kK + st * L::kTileBytes;
+        // FP8: addresses pass through an opaque move, so each call site
+        // derives its descriptors in place instead of holding them across the
+        // loops (its MMA thread also issues the next item's early S0).
+        const uint32_t q_addr = kEarlyS0 ? opaque_u32(base + (t ? L::kQ1 : L::kQ0)) : base + (t ? L::kQ1 : L::kQ0);
+        const uint32_t k_addr =
+            kEarlyS0 ? opaque_u32(base + L::kK + st * L::kTileBytes) : base + L::kK + st * L::kTileBytes;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(t) * 128u;
 #pragma unroll
         for (int kk = 0; kk < kSSteps; ++kk) {
@@ -741,7 +789,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mma_commit(bar(L::kBarSFull + t));
       };
       auto issue_pv = [&](int t, int st, bool accumulate) {
-        const uint32_t v_addr = base + L::kV + st * L::kTileBytes;
+        const uint32_t v_addr =
+            kEarlyS0 ? opaque_u32(base + L::kV + st * L::kTileBytes) : base + L::kV + st * L::kTileBytes;
         const uint32_t p_tmem = tmem + static_cast<uint32_t>(t) * 128u;
         const uint32_t o_tmem = tmem + L::kColO + static_cast<uint32_t>(t * D);
 #pragma unroll
@@ -758,22 +807,28 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if constexpr (SPARSE) {
         // Block-sparse: each query tile visits an arbitrary set of KV tiles;
         // the item walks their union.
-        uint32_t q_cnt = 0;  // items whose Q was loaded (every item except fully masked block-sparse ones)
+        uint32_t q_cnt[2] = {0u, 0u};  // loads of Q tile t waited for (fully masked items load none)
         for (int r = 0; ok; ++r) {
           // The item's tile list, from the lister warp (length -1: no items left).
           const int buf = r & 1;
           if (!(ok = mbar_wait(bar(L::kBarListFull + buf), static_cast<uint32_t>(r >> 1) & 1u, kErrWaitList))) break;
           const volatile uint16_t* const tl =
               reinterpret_cast<const volatile uint16_t*>(smem + L::kSeq + L::kTileList + buf * L::kTileListBytes);
-          const int n_u = reinterpret_cast<const volatile int*>(smem + L::kSeq + L::kTileCount)[buf];
-          if (n_u < 0) break;
+          const int n_raw = reinterpret_cast<const volatile int*>(smem + L::kSeq + L::kTileCount)[buf];
+          if (n_raw < 0) break;
+          const int n_u = n_raw & 0xffff;
+          const bool has1 = (n_raw >> 30) & 1;
           if (n_u == 0) {  // nothing to compute (the epilogue writes zeros)
             mbar_arrive(bar(L::kBarListEmpty + buf));
             continue;
           }
           auto on = [&](int t, int e) { return ((e >> (8 + t)) & 1) != 0; };
-          if (!(ok = mbar_wait(bar(L::kBarQFull), q_cnt & 1u, kErrWaitQ))) break;
-          ++q_cnt;
+          if (!(ok = mbar_wait(bar(L::kBarQFull + 0), q_cnt[0] & 1u, kErrWaitQ))) break;
+          ++q_cnt[0];
+          if (has1) {
+            if (!(ok = mbar_wait(bar(L::kBarQFull + 1), q_cnt[1] & 1u, kErrWaitQ))) break;
+            ++q_cnt[1];
+          }
           {
             const int st = kv_it % NS;
             if (!(ok = mbar_wait(bar(L::kBarKFull + st), static_cast<uint32_t>(kv_it / NS) & 1u, kErrWaitKFull)))
@@ -782,7 +837,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             if (on(0, tl[0])) issue_s(0, st);
             if (on(1, tl[0])) issue_s(1, st);
             mma_commit(bar(L::kBarKEmpty + st));
-            if (n_u == 1) mma_commit(bar(L::kBarQEmpty));  // last S of the item
+            if (n_u == 1) {  // last S of the item
+              mma_commit(bar(L::kBarQEmpty + 0));
+              if (has1) mma_commit(bar(L::kBarQEmpty + 1));
+            }
           }
           // First and last KV tile of each query tile: where O_t starts (after
           // the epilogue released it) and where it is final.
@@ -842,7 +900,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             mma_commit(bar(L::kBarVEmpty + st));
             if (more) mma_commit(bar(L::kBarKEmpty + st1));
-            if (u + 2 == n_u) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
+            if (u + 2 == n_u) {  // the item's last S MMAs were just issued
+              mma_commit(bar(L::kBarQEmpty + 0));
+              if (has1) mma_commit(bar(L::kBarQEmpty + 1));
+            }
           }
           if (!ok) break;
           kv_it += u;
@@ -850,18 +911,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       } else {
         // Dense: query tile t visits the contiguous range [lo(t), hi(t)).
+        uint32_t q_cnt[2] = {0u, 0u};  // loads of Q tile t waited for
+        bool s0_early = false;         // this item's first S0 was issued during the previous item
         for (int r = 0; ok && prefill_item<CAUSAL, WINDOW, PAGED, SPARSE>(r, p, it, sq); ++r) {
-          if (!(ok = mbar_wait(bar(L::kBarQFull), static_cast<uint32_t>(r) & 1u, kErrWaitQ))) break;
+          // Every item's query tile 0 starts at the item's first KV tile, so
+          // only the next item's existence matters for the early S0 below.
+          const bool have_nx = kEarlyS0 && prefill_item_exists<PAGED>(r + 1, p, sq);
           const int nkv = it.je - it.jb;
           {
             const int st = kv_it % NS;
-            if (!(ok = mbar_wait(bar(L::kBarKFull + st), static_cast<uint32_t>(kv_it / NS) & 1u, kErrWaitKFull)))
-              break;
-            tc_fence_after();
-            if (it.active(0, it.jb)) issue_s(0, st);
-            if (it.active(1, it.jb)) issue_s(1, st);
+            if (!s0_early) {
+              if (!(ok = mbar_wait(bar(L::kBarQFull + 0), q_cnt[0] & 1u, kErrWaitQ))) break;
+              ++q_cnt[0];
+              if (!(ok = mbar_wait(bar(L::kBarKFull + st), static_cast<uint32_t>(kv_it / NS) & 1u, kErrWaitKFull)))
+                break;
+              tc_fence_after();
+              if (it.active(0, it.jb)) issue_s(0, st);
+            }
+            s0_early = false;
+            if (it.has(1)) {
+              if (!(ok = mbar_wait(bar(L::kBarQFull + 1), q_cnt[1] & 1u, kErrWaitQ))) break;
+              ++q_cnt[1];
+              tc_fence_after();
+              if (it.active(1, it.jb)) issue_s(1, st);
+            }
             mma_commit(bar(L::kBarKEmpty + st));
-            if (nkv == 1) mma_commit(bar(L::kBarQEmpty));  // last S of the item: Q may be replaced
+            // A query tile's Q may be replaced once its last S is issued.
+            if (it.hi0 - 1 == it.jb) mma_commit(bar(L::kBarQEmpty + 0));
+            if (it.has(1) && it.hi1 - 1 == it.jb) mma_commit(bar(L::kBarQEmpty + 1));
           }
           for (int j = it.jb; j < it.je && ok; ++j) {
             const int g = kv_it + (j - it.jb);
@@ -887,6 +964,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 k_ready = true;
                 tc_fence_after();
                 issue_s(0, st1);
+                if (j + 2 == it.hi0) mma_commit(bar(L::kBarQEmpty + 0));  // Q0's last S
               }
             }
             if (it.active(1, j)) {
@@ -908,10 +986,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               if (!k_ready && !(ok = mbar_wait(bar(L::kBarKFull + st1), ph1, kErrWaitKFull))) break;
               tc_fence_after();
               issue_s(1, st1);
+              if (j + 2 == it.hi1) mma_commit(bar(L::kBarQEmpty + 1));  // Q1's last S
             }
             mma_commit(bar(L::kBarVEmpty + st));
             if (j + 1 < it.je) mma_commit(bar(L::kBarKEmpty + st1));
-            if (j + 2 == it.je) mma_commit(bar(L::kBarQEmpty));  // the item's last S MMAs were just issued
+            if (kEarlyS0 && j + 1 == it.hi0 && have_nx) {
+              // Q0's work of this item is all issued (its last P V just now, so
+              // P0 is consumed).  If the next item's Q0 and first K tile have
+              // already landed, issue its first S0 now: query tile 0 then
+              // starts the next item while query tile 1 finishes this one.
+              // Only tests: nothing here waits.
+              const int gn = kv_it + nkv;
+              const int stn = gn % NS;
+              if (mbar_test(bar(L::kBarQFull + 0), q_cnt[0] & 1u) &&
+                  mbar_test(bar(L::kBarKFull + stn), static_cast<uint32_t>(gn / NS) & 1u)) {
+                ++q_cnt[0];
+                tc_fence_after();
+                issue_s(0, stn);
+                s0_early = true;
+              }
+            }
           }
           if (!ok) break;
           kv_it += nkv;
@@ -975,7 +1069,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tl[pos++] = static_cast<uint16_t>(e);
           }
         }
-        if (lane == 0) reinterpret_cast<volatile int*>(smem + L::kSeq + L::kTileCount)[buf] = n_u;
+        // Length, and bit 30: the item has a second query tile (its Q1 is loaded).
+        if (lane == 0)
+          reinterpret_cast<volatile int*>(smem + L::kSeq + L::kTileCount)[buf] =
+              n_u < 0 ? n_u : (n_u | (it.has(1) ? 1 << 30 : 0));
         __threadfence_block();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::kBarListFull + buf));  // release: the entries above are visible
