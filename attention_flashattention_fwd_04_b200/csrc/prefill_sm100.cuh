@@ -756,10 +756,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t idesc_qk =
           FP8 ? make_idesc_e4m3(128, 128, false, false) : make_idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = FP8 ? make_idesc_e4m3(128, D, false, true) : make_idesc_bf16(128, D, false, true);
-      // The next item's first S0 is issued early in the FP8 kernel, whose
-      // shorter MMA leg leaves the tile-0 softmax waiting at item boundaries;
-      // in the bf16 kernels the extra issue work costs more than it saves.
-      constexpr bool kEarlyS0 = FP8;
+      // The next item's first S0 is issued during the current item's last
+      // tile (below), so query tile 0 starts the next item while query tile 1
+      // finishes this one.  Windowed items are long and equal: they skip it.
+      constexpr bool kEarlyS0 = !WINDOW;
       // Every MMA takes 32 bytes of its K dimension: 16 bf16 or 32 e4m3.
       constexpr int kSSteps = D * L::kElemBytes / 32;     // S = Q K^T over the head dim
       constexpr int kPvKeys = 32 / L::kElemBytes;         // keys per P V step
@@ -768,13 +768,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t p_cnt[2] = {0u, 0u};
       uint32_t o_cnt[2] = {0u, 0u};  // items whose O_t has been completed
       bool ok = true;
-      auto issue_s = [&](int t, int st) {
-        // FP8: addresses pass through an opaque move, so each call site
-        // derives its descriptors in place instead of holding them across the
-        // loops (its MMA thread also issues the next item's early S0).
-        const uint32_t q_addr = kEarlyS0 ? opaque_u32(base + (t ? L::kQ1 : L::kQ0)) : base + (t ? L::kQ1 : L::kQ0);
-        const uint32_t k_addr =
-            kEarlyS0 ? opaque_u32(base + L::kK + st * L::kTileBytes) : base + L::kK + st * L::kTileBytes;
+      auto issue_s = [&](int t, int st, bool opaque = false) {
+        // Addresses through an opaque move make a call site derive its
+        // descriptors in place instead of holding them across the loops: the
+        // early S0's site always (it would otherwise widen the hoisted set
+        // past the MMA thread's registers), every site in the FP8 kernel.
+        const bool op = FP8 || opaque;
+        const uint32_t q_addr = op ? opaque_u32(base + (t ? L::kQ1 : L::kQ0)) : base + (t ? L::kQ1 : L::kQ0);
+        const uint32_t k_addr = op ? opaque_u32(base + L::kK + st * L::kTileBytes) : base + L::kK + st * L::kTileBytes;
         const uint32_t d_tmem = tmem + static_cast<uint32_t>(t) * 128u;
 #pragma unroll
         for (int kk = 0; kk < kSSteps; ++kk) {
@@ -789,8 +790,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mma_commit(bar(L::kBarSFull + t));
       };
       auto issue_pv = [&](int t, int st, bool accumulate) {
-        const uint32_t v_addr =
-            kEarlyS0 ? opaque_u32(base + L::kV + st * L::kTileBytes) : base + L::kV + st * L::kTileBytes;
+        const uint32_t v_addr = FP8 ? opaque_u32(base + L::kV + st * L::kTileBytes) : base + L::kV + st * L::kTileBytes;
         const uint32_t p_tmem = tmem + static_cast<uint32_t>(t) * 128u;
         const uint32_t o_tmem = tmem + L::kColO + static_cast<uint32_t>(t * D);
 #pragma unroll
@@ -1002,7 +1002,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                   mbar_test(bar(L::kBarKFull + stn), static_cast<uint32_t>(gn / NS) & 1u)) {
                 ++q_cnt[0];
                 tc_fence_after();
-                issue_s(0, stn);
+                issue_s(0, stn, true);
                 s0_early = true;
               }
             }
