@@ -220,3 +220,24 @@ def _bias(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=2, N=300
 ])
 def test_attn_fwd_bias_rejects(lib, kw, code):
     assert _bias(lib, **kw) == code
+
+
+def test_pack_block_mask_bit_layout():
+    """The binding's packer (marshalling only, runs wherever the tensor is):
+    bit j % 64 of word j / 64 set iff key block j is kept, bit 63 included."""
+    import numpy as np
+    import torch
+    from attention_flashattention_fwd_04_b200 import api
+    rng = np.random.default_rng(9)
+    for nb in (1, 63, 64, 65, 130, 256):
+        keep = torch.from_numpy(rng.random((2, 3, 4, nb)) < 0.5)
+        keep[0, 0, 0, nb - 1] = True
+        words = api.pack_block_mask(keep)
+        assert words.dtype == torch.int64 and words.shape == (2, 3, 4, -(-nb // 64))
+        u = words.numpy().view(np.uint64)
+        for idx in np.ndindex(2, 3, 4):
+            for j in range(nb):
+                bit = (int(u[idx + (j // 64,)]) >> (j % 64)) & 1
+                assert bit == int(keep[idx + (j,)])
+            for j in range(nb, 64 * u.shape[-1]):          # bits past the last block stay clear
+                assert (int(u[idx + (j // 64,)]) >> (j % 64)) & 1 == 0

@@ -172,3 +172,25 @@ def test_bench_mask_work_accounting():
     # the per-head M makes this prefill HBM-bound at the measured peaks
     peaks = bench.load_peaks()
     assert b / (peaks["hbm_gbs"] * 1e9) > f / (peaks["bf16_tflops"] * 1e12)
+
+
+def test_traffic_records_follow_each_kernels_sources(tmp_path, monkeypatch):
+    """A traffic record counts only while its kernel's own sources are
+    unchanged: records whose hash does not match are dropped."""
+    import bench
+    good = bench.kernel_source_hash("decode_split_kernel")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "ncu_traffic.txt").write_text(
+        "# comment\n"
+        f"kernel=decode_split_kernel bench=paged_decode sha={good} dram_bytes_per_launch=123 read=100 write=23\n"
+        "kernel=prefill_fwd_kernel bench=causal_mha sha=0000000000000000 dram_bytes_per_launch=5 read=4 write=1\n"
+        f"kernel=unknown_kernel bench=x sha={good} dram_bytes_per_launch=7 read=7 write=0\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash",
+                        lambda k=None: good if k == "decode_split_kernel" else "ffffffffffffffff")
+    t = bench.load_traffic()
+    assert t == {("decode_split_kernel", "paged_decode"): 123.0}
+    # every kernel the bench reports has a source set, and every listed file exists
+    for k, files in bench.KERNEL_SOURCE_SETS.items():
+        assert set(files) <= set(bench.KERNEL_SOURCES)
