@@ -500,6 +500,18 @@ def attn_fwd_block_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, kee
     return out, lse
 
 
+def bias_span_ok(bias: torch.Tensor, strides) -> bool:
+    """Whether every element the additive-M kernel reads lies in ``bias``'s
+    storage: each row is read in 16-byte vectors up to the next multiple of 8
+    elements, so the last row's padding must be there too (the C ABI takes a
+    plain pointer and cannot check this)."""
+    N = bias.shape[3]
+    padded = -(-N // 8) * 8
+    last = sum((bias.shape[i] - 1) * strides[i] for i in range(3)) + padded - 1
+    end_bytes = (bias.storage_offset() + last + 1) * bias.element_size()
+    return end_bytes <= bias.untyped_storage().nbytes()
+
+
 def attn_fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: torch.Tensor, causal: bool = False,
                   scale: float | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
                   stream=None):
@@ -526,6 +538,9 @@ def attn_fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: torch
     if N > 1 and bias.stride(3) != 1:
         raise ValueError("bias rows must be contiguous")
     strides = [0 if bias.shape[i] == 1 else bias.stride(i) for i in range(3)]
+    if not bias_span_ok(bias, strides):
+        raise ValueError("bias rows must be padded to a multiple of 8 elements within the tensor's storage "
+                         "(e.g. a [..., :N] view of a buffer whose last dimension is rounded up to 8)")
     if scale is None:
         scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
     if out is None:

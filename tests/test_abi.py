@@ -241,3 +241,21 @@ def test_pack_block_mask_bit_layout():
                 assert bit == int(keep[idx + (j,)])
             for j in range(nb, 64 * u.shape[-1]):          # bits past the last block stay clear
                 assert (int(u[idx + (j // 64,)]) >> (j % 64)) & 1 == 0
+
+
+def test_bias_span_check():
+    """The binding refuses an M whose padded rows would reach past its storage."""
+    import torch
+    from attention_flashattention_fwd_04_b200 import api
+    ok = torch.zeros(1, 2, 5, 16, dtype=torch.bfloat16)[..., :13]          # rows padded to 16
+    assert api.bias_span_ok(ok, [0, ok.stride(1), ok.stride(2)])
+    tight = torch.zeros(1, 2, 5, 13, dtype=torch.bfloat16)                 # 13-element rows, no padding
+    assert not api.bias_span_ok(tight, [0, tight.stride(1), tight.stride(2)])
+    row = torch.zeros(2, 1, 1, 601, dtype=torch.bfloat16)                  # key-padding row, 601 not padded
+    assert not api.bias_span_ok(row, [row.stride(0), 0, 0])
+    row = torch.zeros(2, 1, 1, 608, dtype=torch.bfloat16)[..., :601]
+    assert api.bias_span_ok(row, [row.stride(0), 0, 0])
+    mult8 = torch.zeros(1, 1, 7, 64, dtype=torch.bfloat16)                 # N a multiple of 8: no padding needed
+    assert api.bias_span_ok(mult8, [0, 0, mult8.stride(2)])
+    off = torch.zeros(1, 1, 1, 24, dtype=torch.bfloat16)[..., 8:]          # a view ending exactly at the storage end
+    assert api.bias_span_ok(off, [0, 0, 0])
