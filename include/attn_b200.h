@@ -43,7 +43,7 @@ typedef enum attn_status {
   ATTN_ERR_SHAPE = 2,       /* a size is out of range or inconsistent */
   ATTN_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
   ATTN_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required */
-  ATTN_ERR_UNSUPPORTED = 5, /* valid input this build has no kernel for */
+  ATTN_ERR_UNSUPPORTED = 5, /* valid input the library has no kernel for */
   ATTN_ERR_LAUNCH = 6,      /* CUDA refused the launch (see attn_last_cuda_error) */
   ATTN_ERR_DEVICE = 7       /* a kernel recorded a runtime error (attn_device_status) */
 } attn_status;
