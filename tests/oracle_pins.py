@@ -563,6 +563,12 @@ def pin_bias_sdpa(o):
                 ref_lse = torch.logsumexp(0.3 * (tq @ tk.T) + tm, -1)
                 assert np.max(np.abs(out[b, h][rows.numpy()] - ref.numpy())) < 1e-12
                 assert np.max(np.abs(lse[b, h][rows.numpy()] - ref_lse[rows].numpy())) < 1e-12
+                # rows M leaves without a finite score (head 1, rows 0..2 under the causal
+                # mask): O = 0, LSE = -inf
+                empty = ~rows.numpy()
+                if causal and h == 1:
+                    assert empty[:3].all()
+                assert np.all(out[b, h][empty] == 0.0) and np.all(np.isneginf(lse[b, h][empty]))
 
 
 def pin_bias_invariants(o):
