@@ -29,3 +29,19 @@ def test_reference_arm_line(workload):
     assert line["config"]["workload"]
     if workload != "tiny":
         assert "mask" in line["config"]["workload"] or "M per head" in line["config"]["workload"]
+
+
+def test_reference_arm_under_two_ranks():
+    """Launched on 2 ranks, rank 0 alone runs the oracle and prints the line
+    (n_gpus = 2); rank 1 exits 0 without work or output."""
+    base = dict(os.environ, CUDA_VISIBLE_DEVICES="", WORLD_SIZE="2", LOCAL_RANK="0")
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny", "--gpus", "2", "--steps", "1",
+           "--warmup", "3"]
+    r1 = subprocess.run(cmd, cwd=ROOT, env=dict(base, RANK="1", LOCAL_RANK="1"), capture_output=True, text=True,
+                        timeout=600)
+    assert r1.returncode == 0, r1.stderr[-2000:]
+    assert r1.stdout.strip() == ""
+    r0 = subprocess.run(cmd, cwd=ROOT, env=dict(base, RANK="0"), capture_output=True, text=True, timeout=600)
+    assert r0.returncode == 0, r0.stderr[-2000:]
+    line = json.loads(r0.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
