@@ -143,9 +143,12 @@ int attn_fwd_bias(const attn_bf16* q, const attn_bf16* k, const attn_bf16* v, at
  * attn_fwd_fp8 -- attn_fwd with e4m3 inputs (OCP FP8 E4M3 codes, one byte
  * each, same [B, H, N, d] layouts): the attention of q * q_descale,
  * k * k_descale and v * v_descale, the FP8 tensor-core path of FlashAttention
- * v3 (the anylearn.cc lesson's FA v3 section).  Q K^T and P V run on the FP8
- * tensor cores with fp32 accumulation; P is rounded to e4m3 (scaled by 2^8)
- * before P V, the row sums and LSE use P unrounded.  o is bf16, lse fp32.
+ * v3 ("Kernel Fusion and Custom Kernels", ai.zenoagi.com, section 3
+ * "FlashAttention: The Milestone of Fusion", under "v3 (2024,
+ * H100-Exclusive)": Q K and P V computed in FP8 for twice the tensor-core
+ * rate).  Q K^T and P V run on the FP8 tensor cores with fp32 accumulation;
+ * P is rounded to e4m3 (scaled by 2^8) before P V, the row sums and LSE use
+ * P unrounded.  o is bf16, lse fp32.
  * d must be 128 (ATTN_ERR_UNSUPPORTED for 64); the descales finite and > 0.
  * Error behaviour as attn_fwd.
  */

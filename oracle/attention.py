@@ -44,9 +44,10 @@ Readings where the pages are silent (each is restated where it is used):
 * additive M (the attention equation's M in general: any finite values, -inf
   allowed): a [B|1, Hq|1, N, N] array in natural-log units added to the
   scaled scores, S = scale * q k^T + M, on top of the causal mask.
-* FP8 inputs (the anylearn.cc lesson's FA v3 section: Q K^T and P V computed
-  in FP8): Q, K, V arrive as e4m3 codes with one descale factor per tensor;
-  the operation is attention over the decoded values times their descales
+* FP8 inputs ("Kernel Fusion and Custom Kernels", ai.zenoagi.com, section 3
+  "FlashAttention: The Milestone of Fusion", under "v3 (2024, H100-Exclusive)":
+  Q K^T and P V computed in FP8): Q, K, V arrive as e4m3 codes with one
+  descale factor per tensor; the operation is attention over the decoded values times their descales
   (e4m3: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals at
   exponent field 0, no infinities, the all-ones code NaN).
 * appending to the cache / chunked prefill ("Operator Fusion" section: the
