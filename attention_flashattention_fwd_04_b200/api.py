@@ -9,6 +9,7 @@ the library is missing or a call fails, this module raises.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 import re
 
@@ -122,10 +123,10 @@ def _stream_handle(stream) -> int:
     return s.cuda_stream
 
 
-def _require(t: torch.Tensor, name: str, dtype, ndim: int):
+def _require(t: torch.Tensor, name: str, dtype, ndim: int, cuda: bool = True):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if not t.is_cuda:
+    if cuda and not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
@@ -135,6 +136,21 @@ def _require(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _on_first_tensor_device(fn):
+    """Runs a wrapper with its first tensor argument's CUDA device current, so
+    that the stream it takes and any output it allocates belong to that
+    device (the kernels run on the current device)."""
+    @functools.wraps(fn)
+    def wrapped(*args, **kwargs):
+        first = next((a for a in args if isinstance(a, torch.Tensor)), None)
+        if first is None or not first.is_cuda:
+            return fn(*args, **kwargs)  # the wrapper's own checks reject it
+        with torch.cuda.device(first.device):
+            return fn(*args, **kwargs)
+    return wrapped
+
+
+@_on_first_tensor_device
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True,
              scale: float | None = None, out: torch.Tensor | None = None,
              lse: torch.Tensor | None = None, stream=None, window_left: int | None = None):
@@ -178,6 +194,42 @@ def paged_attn_decode_workspace_bytes(num_seqs: int, Hq: int, d: int, max_pages:
     return int(lib().paged_attn_decode_workspace_bytes(num_seqs, Hq, d, max_pages, page_size))
 
 
+def _decode_args(q, k_pool, v_pool, block_table, seq_lens, out=None, lse=None):
+    """Checks shared by the paged-decode wrappers, made before any CUDA call
+    (the C layer sees only pointers, so a short v_pool, block_table or
+    seq_lens would be read past its end): dtypes, ranks, contiguity and
+    consistent shapes first, then that every tensor is on q's CUDA device.
+    Returns (S, Hq, d, num_pages, page_size, Hkv, max_pages)."""
+    named = [(q, "q", torch.bfloat16, 3), (k_pool, "k_pool", torch.bfloat16, 4),
+             (v_pool, "v_pool", torch.bfloat16, 4), (block_table, "block_table", torch.int32, 2),
+             (seq_lens, "seq_lens", torch.int32, 1)]
+    if out is not None:
+        named.append((out, "out", torch.bfloat16, 3))
+    if lse is not None:
+        named.append((lse, "lse", torch.float32, 2))
+    for t, name, dt, nd in named:
+        _require(t, name, dt, nd, cuda=False)
+    S, Hq, d = q.shape
+    num_pages, page_size, Hkv, dk = k_pool.shape
+    if dk != d:
+        raise ValueError(f"k_pool's head dim {dk} does not match q's {d}")
+    if v_pool.shape != k_pool.shape:
+        raise ValueError(f"v_pool shape {tuple(v_pool.shape)} differs from k_pool's {tuple(k_pool.shape)}")
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError(f"block_table {tuple(block_table.shape)} / seq_lens {tuple(seq_lens.shape)} do not "
+                         f"have one row per sequence ({S})")
+    if out is not None and out.shape != q.shape:
+        raise ValueError(f"out shape {tuple(out.shape)} differs from q's {tuple(q.shape)}")
+    if lse is not None and lse.shape != (S, Hq):
+        raise ValueError(f"lse shape {tuple(lse.shape)} is not ({S}, {Hq})")
+    for t, name, _, _ in named:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
+    return S, Hq, d, num_pages, page_size, Hkv, block_table.shape[1]
+
+
 def paged_attn_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
                       block_table: torch.Tensor, seq_lens: torch.Tensor, scale: float | None = None,
                       workspace: torch.Tensor | None = None, out: torch.Tensor | None = None,
@@ -188,31 +240,24 @@ def paged_attn_decode(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tenso
     block_table [S,max_pages] int32; seq_lens [S] int32 (all on the GPU).
     Returns (o [S,Hq,d] bf16, lse [S,Hq] fp32).
     """
-    _require(q, "q", torch.bfloat16, 3)
-    _require(k_pool, "k_pool", torch.bfloat16, 4)
-    _require(v_pool, "v_pool", torch.bfloat16, 4)
-    _require(block_table, "block_table", torch.int32, 2)
-    _require(seq_lens, "seq_lens", torch.int32, 1)
-    S, Hq, d = q.shape
-    num_pages, page_size, Hkv, dk = k_pool.shape
-    if dk != d or v_pool.shape != k_pool.shape:
-        raise ValueError("pool shapes do not match q")
-    if block_table.shape[0] != S or seq_lens.shape[0] != S:
-        raise ValueError("block_table / seq_lens do not match the number of sequences")
-    max_pages = block_table.shape[1]
+    S, Hq, d, num_pages, page_size, Hkv, max_pages = _decode_args(q, k_pool, v_pool, block_table, seq_lens,
+                                                                  out, lse)
     if scale is None:
         scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
-    need = paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, page_size)
-    if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
-    rc = lib().paged_attn_decode(
-        q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
-        page_size, out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages, float(scale),
-        workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    with torch.cuda.device(q.device):
+        need = paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, page_size)
+        if workspace is None:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        elif not workspace.is_cuda or workspace.device != q.device:
+            raise ValueError(f"workspace must be on {q.device}")
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+        rc = lib().paged_attn_decode(
+            q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+            page_size, out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages, float(scale),
+            workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_handle(stream))
     _check(rc, "paged_attn_decode")
     return out, lse
 
@@ -226,25 +271,21 @@ def paged_attn_decode_noalloc(q: torch.Tensor, k_pool: torch.Tensor, v_pool: tor
     to a 48 MiB array built into the library, shared by all calls on a
     device: calls that can overlap on the GPU must not use it concurrently.
     """
-    _require(q, "q", torch.bfloat16, 3)
-    _require(k_pool, "k_pool", torch.bfloat16, 4)
-    _require(v_pool, "v_pool", torch.bfloat16, 4)
-    _require(block_table, "block_table", torch.int32, 2)
-    _require(seq_lens, "seq_lens", torch.int32, 1)
-    S, Hq, d = q.shape
-    num_pages, page_size, Hkv, _ = k_pool.shape
+    S, Hq, d, num_pages, page_size, Hkv, max_pages = _decode_args(q, k_pool, v_pool, block_table, seq_lens,
+                                                                  out, lse)
     if scale is None:
         scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
-    rc = lib().paged_attn_decode_noalloc(
-        q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
-        page_size, out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, block_table.shape[1], num_pages,
-        float(scale), _stream_handle(stream))
+    with torch.cuda.device(q.device):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+        rc = lib().paged_attn_decode_noalloc(
+            q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+            page_size, out.data_ptr(), lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages,
+            float(scale), _stream_handle(stream))
     if rc == 4:
-        need = paged_attn_decode_workspace_bytes(S, Hq, d, block_table.shape[1], page_size)
+        need = paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, page_size)
         raise AttnError(rc, f"paged_attn_decode_noalloc: needs {need} bytes of scratch, "
                             f"more than the built-in {NOALLOC_SCRATCH_BYTES}")
     _check(rc, "paged_attn_decode_noalloc")
@@ -261,35 +302,36 @@ class DecodeGraph:
     """
 
     def __init__(self, q, k_pool, v_pool, block_table, seq_lens, scale=None, workspace=None, out=None, lse=None):
-        for t, name, dt, nd in ((q, "q", torch.bfloat16, 3), (k_pool, "k_pool", torch.bfloat16, 4),
-                                (v_pool, "v_pool", torch.bfloat16, 4), (block_table, "block_table", torch.int32, 2),
-                                (seq_lens, "seq_lens", torch.int32, 1)):
-            _require(t, name, dt, nd)
-        S, Hq, d = q.shape
-        num_pages, page_size, Hkv, _ = k_pool.shape
-        max_pages = block_table.shape[1]
+        self._handle = None
+        S, Hq, d, num_pages, page_size, Hkv, max_pages = _decode_args(q, k_pool, v_pool, block_table, seq_lens,
+                                                                      out, lse)
         if scale is None:
             scale = float(torch.tensor(d ** -0.5, dtype=torch.float32))
-        need = paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, page_size)
-        self.workspace = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8,
-                                                                             device=q.device)
-        self.out = out if out is not None else torch.empty_like(q)
-        self.lse = lse if lse is not None else torch.empty((S, Hq), dtype=torch.float32, device=q.device)
-        self._keep = (q, k_pool, v_pool, block_table, seq_lens)
-        handle = ctypes.c_void_p()
-        rc = lib().paged_attn_decode_graph_create(
-            q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
-            page_size, self.out.data_ptr(), self.lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages,
-            float(scale), self.workspace.data_ptr(), self.workspace.numel() * self.workspace.element_size(),
-            ctypes.byref(handle))
+        self.device = q.device
+        with torch.cuda.device(q.device):
+            need = paged_attn_decode_workspace_bytes(S, Hq, d, max_pages, page_size)
+            if workspace is not None and (not workspace.is_cuda or workspace.device != q.device):
+                raise ValueError(f"workspace must be on {q.device}")
+            self.workspace = workspace if workspace is not None else torch.empty(
+                max(need, 16), dtype=torch.uint8, device=q.device)
+            self.out = out if out is not None else torch.empty_like(q)
+            self.lse = lse if lse is not None else torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+            self._keep = (q, k_pool, v_pool, block_table, seq_lens)
+            handle = ctypes.c_void_p()
+            rc = lib().paged_attn_decode_graph_create(
+                q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), block_table.data_ptr(), seq_lens.data_ptr(),
+                page_size, self.out.data_ptr(), self.lse.data_ptr(), S, Hq, Hkv, d, max_pages, num_pages,
+                float(scale), self.workspace.data_ptr(), self.workspace.numel() * self.workspace.element_size(),
+                ctypes.byref(handle))
         _check(rc, "paged_attn_decode_graph_create")
         self._handle = handle
 
     def launch(self, stream=None):
         if self._handle is None:
             raise RuntimeError("DecodeGraph is closed")
-        _check(lib().paged_attn_decode_graph_launch(self._handle, _stream_handle(stream)),
-               "paged_attn_decode_graph_launch")
+        with torch.cuda.device(self.device):
+            rc = lib().paged_attn_decode_graph_launch(self._handle, _stream_handle(stream))
+        _check(rc, "paged_attn_decode_graph_launch")
         return self.out, self.lse
 
     def close(self):
@@ -328,6 +370,7 @@ def _paged_chunk_args(k_pool, v_pool, block_table, cu_seqlens_q, seq_lens):
     return S, num_pages, page_size, Hkv, d, block_table.shape[1]
 
 
+@_on_first_tensor_device
 def paged_kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor,
                     block_table: torch.Tensor, cu_seqlens_q: torch.Tensor, seq_lens: torch.Tensor, stream=None):
     """Write each sequence's new K/V rows (packed [total_q, Hkv, d] bf16,
@@ -357,6 +400,7 @@ def _prefill_outputs(q, out, lse):
     return out, lse
 
 
+@_on_first_tensor_device
 def paged_prefill(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, block_table: torch.Tensor,
                   cu_seqlens_q: torch.Tensor, seq_lens: torch.Tensor, causal: bool = True,
                   scale: float | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
@@ -381,6 +425,7 @@ def paged_prefill(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, b
     return out, lse
 
 
+@_on_first_tensor_device
 def paged_prefill_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, k_pool: torch.Tensor,
                          v_pool: torch.Tensor, block_table: torch.Tensor, cu_seqlens_q: torch.Tensor,
                          seq_lens: torch.Tensor, causal: bool = True, scale: float | None = None,
@@ -407,6 +452,7 @@ def paged_prefill_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tens
     return out, lse
 
 
+@_on_first_tensor_device
 def attn_fwd_fp8(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, scale: float | None = None,
                  q_descale: float = 1.0, k_descale: float = 1.0, v_descale: float = 1.0,
                  out: torch.Tensor | None = None, lse: torch.Tensor | None = None, stream=None):
@@ -454,6 +500,7 @@ def pack_block_mask(keep: torch.Tensor) -> torch.Tensor:
     return (bits * weights).sum(-1)  # bit 63 wraps to the sign bit: the same 64 bits
 
 
+@_on_first_tensor_device
 def attn_fwd_block_sparse(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, keep: torch.Tensor,
                           causal: bool = True, scale: float | None = None, out: torch.Tensor | None = None,
                           lse: torch.Tensor | None = None, stream=None):
@@ -512,6 +559,7 @@ def bias_span_ok(bias: torch.Tensor, strides) -> bool:
     return end_bytes <= bias.untyped_storage().nbytes()
 
 
+@_on_first_tensor_device
 def attn_fwd_bias(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, bias: torch.Tensor, causal: bool = False,
                   scale: float | None = None, out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
                   stream=None):

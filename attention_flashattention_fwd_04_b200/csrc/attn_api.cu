@@ -316,6 +316,22 @@ int validate_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16
 
 }  // namespace
 
+// Library-internal (hidden, not part of the C ABI): used by the no-alloc
+// entry point in attn_noalloc.cu, which is built as a separate file.
+// attn_internal_validate_decode runs paged_attn_decode's host-side checks
+// (no CUDA call); attn_internal_cuda_failure records a CUDA error for
+// attn_last_cuda_error and returns ATTN_ERR_LAUNCH.
+__attribute__((visibility("hidden"))) int attn_internal_validate_decode(
+    const attn_bf16* q, const attn_bf16* k_pool, const attn_bf16* v_pool, const int32_t* block_table,
+    const int32_t* seq_lens, int page_size, attn_bf16* o, float* lse, int num_seqs, int Hq, int Hkv, int d,
+    int max_pages, int num_pages, float scale, void* workspace, size_t workspace_bytes) {
+  DecodePlan pl;
+  return validate_decode(q, k_pool, v_pool, block_table, seq_lens, page_size, o, lse, num_seqs, Hq, Hkv, d,
+                         max_pages, num_pages, scale, workspace, workspace_bytes, &pl);
+}
+
+__attribute__((visibility("hidden"))) int attn_internal_cuda_failure(cudaError_t e) { return fail_cuda(e); }
+
 extern "C" {
 
 

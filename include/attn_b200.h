@@ -224,17 +224,26 @@ int paged_attn_decode(const attn_bf16* q, const attn_bf16* k_pool, const attn_bf
  * whose memory pool has already reserved everything.  Such callers pass the
  * same arguments as to paged_attn_decode minus the workspace, and the split
  * partials go to a fixed array of ATTN_NOALLOC_SCRATCH_BYTES compiled into
- * the library.  This call itself never allocates or frees device memory.
+ * the library.  This call never calls cudaMalloc, cudaFree or any other
+ * allocating routine.
  *
  * - Every GPU on which the library's device code is loaded keeps that array
- *   (48 MiB) until the process exits.
+ *   (48 MiB) until the process exits.  The CUDA runtime creates it when it
+ *   loads the library's device code on a device; with lazy module loading
+ *   (the default since CUDA 12.2) that happens inside the first call on that
+ *   device, which then fails with ATTN_ERR_LAUNCH (attn_last_cuda_error()
+ *   names the CUDA error, e.g. out of memory) if the device has no room left.
+ *   Make one warm-up call at start-up, before memory is handed out.
  * - Limit: sizes whose paged_attn_decode_workspace_bytes() exceed
  *   ATTN_NOALLOC_SCRATCH_BYTES are refused with ATTN_ERR_WORKSPACE before any
- *   CUDA call.  (The 64-sequence, 32-head, 8192-token-table workload needs
- *   33.8 MB.)
- * - The first call with a given device current looks up the array's device
- *   address (cudaGetSymbolAddress); make that first call before any stream
- *   capture on that device.
+ *   CUDA call, after the same argument checks as paged_attn_decode (a bad
+ *   argument is reported as itself).  (The 64-sequence, 32-head,
+ *   8192-token-table workload needs 33.8 MB.)
+ * - The first call in each CUDA context of a device looks up the array's
+ *   device address (cudaGetSymbolAddress) and caches it under the context's
+ *   id; after a device reset the next call looks it up again.  Make the first
+ *   call on a device (and the first after a reset) before any stream capture
+ *   on that device.
  * - All calls on a device share the one array and it keeps whatever the last
  *   call left there (nothing in it needs to start at zero).  Calls whose
  *   kernels can overlap on the GPU (different streams, or different host

@@ -99,6 +99,39 @@ def test_python_binding_refuses_cpu_tensors(lib):
         api.attn_fwd(q, q, q)
 
 
+def _decode_tensors(**bad):
+    import torch
+    S, Hq, Hkv, d, pages, ps, mp = 3, 8, 2, 128, 10, 16, 4
+    t = dict(q=torch.zeros(S, Hq, d, dtype=torch.bfloat16),
+             k_pool=torch.zeros(pages, ps, Hkv, d, dtype=torch.bfloat16),
+             v_pool=torch.zeros(pages, ps, Hkv, d, dtype=torch.bfloat16),
+             block_table=torch.zeros(S, mp, dtype=torch.int32),
+             seq_lens=torch.ones(S, dtype=torch.int32))
+    t.update(bad)
+    return t
+
+
+@pytest.mark.parametrize("wrapper", ["paged_attn_decode", "paged_attn_decode_noalloc", "DecodeGraph"])
+@pytest.mark.parametrize("bad, what", [
+    ("v_pool", "v_pool shape"), ("block_table", "one row per sequence"), ("seq_lens", "one row per sequence"),
+    ("k_pool", "head dim")])
+def test_decode_wrappers_refuse_mismatched_shapes_before_any_launch(lib, wrapper, bad, what):
+    # The C layer sees only pointers: a short v_pool, block_table or seq_lens
+    # would be read past its end.  The binding's shape checks come before its
+    # device checks, so they show here on CPU tensors.
+    import torch
+    good = _decode_tensors()
+    shrunk = {"v_pool": good["v_pool"][:-1].contiguous(), "block_table": good["block_table"][:-1].contiguous(),
+              "seq_lens": good["seq_lens"][:-1].contiguous(),
+              "k_pool": torch.zeros(10, 16, 2, 64, dtype=torch.bfloat16)}[bad]
+    t = _decode_tensors(**{bad: shrunk})
+    fn = getattr(api, wrapper)
+    with pytest.raises(ValueError, match=what):
+        fn(t["q"], t["k_pool"], t["v_pool"], t["block_table"], t["seq_lens"], 0.1)
+    with pytest.raises(ValueError, match="CUDA tensor"):  # consistent shapes: then the device check
+        fn(good["q"], good["k_pool"], good["v_pool"], good["block_table"], good["seq_lens"], 0.1)
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(api, "_lib", None)
     monkeypatch.setattr(api, "LIB_PATH", str(tmp_path / "nope.so"))
