@@ -128,7 +128,7 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device, period_s: float = 0.01):
+    def __init__(self, device, period_s: float = 0.001):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
@@ -227,21 +227,23 @@ def prefill_label(c, fp8=False, mask_kind=None) -> str:
         mask += " + " + mask_label(mask_kind)
     return f"{mask} prefill B={c.B} Hq={c.Hq} Hkv={c.Hkv} N={c.N} d={c.d}"
 
-class Step:
-    """Device-resident inputs/outputs for one rank and the calls of one step."""
+class StepSpec:
+    """One rank's workload on the host: configs, seeded inputs and the work
+    the step does (FLOPs, bytes).  Both arms build it, so their `config`
+    objects describe the same workload in the same words."""
 
-    def __init__(self, workload: str, rank: int, device, decode_graph: bool = False):
-        from attention_flashattention_fwd_04_b200 import api
-        self.api = api
-        self.device = device
+    def __init__(self, workload: str, rank: int = 0, mask_tensors: bool = True):
+        self.workload = workload
         self.prefill_cfg = None
         self.decode_cfg = None
         self.chunked_cfg = None
+        self.host = {}      # a step's own inputs (copied in every step by the e2e leg)
         self.resident = {}  # device state that persists across steps: the paged KV caches
         if workload in CHUNKED_WORKLOADS:
             base = W.CHUNKED_CONFIGS[workload]
             self.chunked_cfg = dataclasses.replace(base, seed=shard_seed(base.seed, rank))
         self.fp8 = workload in FP8_WORKLOADS
+        self.descales = None
         self.mask_kind = MASK_WORKLOADS[workload][1] if workload in MASK_WORKLOADS else None
         self.fused_bytes = 0.0  # bytes moved by the prefill kernel itself while it computes
         if workload in PREFILL_WORKLOADS or self.fp8 or self.mask_kind is not None:
@@ -253,10 +255,9 @@ class Step:
             base = W.DECODE_CONFIGS["small_decode" if workload == "small_decode" else "paged_decode"]
             self.decode_cfg = W.DecodeConfig(base.name, base.num_seqs, base.Hq, base.Hkv, base.d, base.page_size,
                                              base.min_len, base.max_len, shard_seed(base.seed, rank))
-        self.host = {}
-        self.dev = {}
         self.flops = 0.0
         self.bytes = 0.0
+        self.decode_inp = None
         if self.prefill_cfg is not None:
             c = self.prefill_cfg
             if self.fp8:
@@ -266,7 +267,8 @@ class Step:
             self.host.update(q=q, k=k, v=v)
             self.flops = W.prefill_flops(c)
             if self.mask_kind is not None:
-                self.host.update(mask_inputs(self.mask_kind, c))
+                if mask_tensors:
+                    self.host.update(mask_inputs(self.mask_kind, c))
                 self.flops, self.fused_bytes = mask_work(self.mask_kind, c)
         if self.decode_cfg is not None:
             c = self.decode_cfg
@@ -288,33 +290,71 @@ class Step:
             self.resident.update(c_k_pool=inp["k_pool"], c_v_pool=inp["v_pool"])
             self.flops = W.chunked_flops(inp["ctx_lens"], inp["q_lens"], c.Hq, c.d)
             self.bytes = W.chunked_append_bytes(inp["q_lens"], c.Hkv, c.d)
+
+    def tensor_peak_tflops(self, peaks) -> float:
+        """Peak for this step's contraction dtype: the measured bf16 GEMM
+        rate, doubled for e4m3 (the nominal dense fp8 / bf16 ratio, 4.5 / 2.25
+        PFLOP/s)."""
+        return peaks["bf16_tflops"] * (2.0 if self.fp8 else 1.0)
+
+    def ideal_seconds(self, peaks) -> float:
+        """Separate kernels add up; within the prefill kernel the tensor work
+        and the bytes it moves overlap, so the slower of the two counts."""
+        prefill = max(self.flops / (self.tensor_peak_tflops(peaks) * 1e12),
+                      self.fused_bytes / (peaks["hbm_gbs"] * 1e9))
+        return prefill + self.bytes / (peaks["hbm_gbs"] * 1e9)
+
+
+class Step(StepSpec):
+    """Device-resident inputs/outputs for one rank and the calls of one step."""
+
+    def __init__(self, workload: str, rank: int, device, decode_graph: bool = False):
+        super().__init__(workload, rank)
+        from attention_flashattention_fwd_04_b200 import api
+        self.api = api
+        self.device = device
+        self.dev = {}
         for name, t in self.host.items():
             self.dev[name] = t.to(device)
         for name, t in self.resident.items():
             self.dev[name] = t.to(device)
-        self._alloc_outputs()
+        self._alloc_outputs(self.dev)
         self.graph = None
         if decode_graph and self.decode_cfg is not None:
-            d = self.dev
-            self.graph = api.DecodeGraph(d["dq"], d["k_pool"], d["v_pool"], d["block_table"], d["seq_lens"],
-                                         self.decode_cfg.scale, workspace=d["ws"], out=d["do"], lse=d["dlse"])
+            self.graph = self.make_graph(self.dev)
 
-    def _alloc_outputs(self):
+    def make_graph(self, d):
+        return self.api.DecodeGraph(d["dq"], d["k_pool"], d["v_pool"], d["block_table"], d["seq_lens"],
+                                    self.decode_cfg.scale, workspace=d["ws"], out=d["do"], lse=d["dlse"])
+
+    OUTPUTS = ("o", "lse", "do", "dlse", "co", "clse")
+
+    def _alloc_outputs(self, d):
         api, dev = self.api, self.device
         if self.prefill_cfg is not None:
-            q = self.dev["q"]
-            self.dev["o"] = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
-            self.dev["lse"] = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+            q = d["q"]
+            d["o"] = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+            d["lse"] = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
         if self.chunked_cfg is not None:
-            q = self.dev["cq"]
-            self.dev["co"] = torch.empty_like(q)
-            self.dev["clse"] = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
+            q = d["cq"]
+            d["co"] = torch.empty_like(q)
+            d["clse"] = torch.empty(q.shape[:2], dtype=torch.float32, device=dev)
         if self.decode_cfg is not None:
             c, inp = self.decode_cfg, self.decode_inp
-            need = api.paged_attn_decode_workspace_bytes(c.num_seqs, c.Hq, c.d, inp["max_pages"], c.page_size)
-            self.dev["ws"] = torch.empty(need, dtype=torch.uint8, device=dev)
-            self.dev["do"] = torch.empty_like(self.dev["dq"])
-            self.dev["dlse"] = torch.empty((c.num_seqs, c.Hq), dtype=torch.float32, device=dev)
+            if "ws" not in d:
+                need = api.paged_attn_decode_workspace_bytes(c.num_seqs, c.Hq, c.d, inp["max_pages"], c.page_size)
+                d["ws"] = torch.empty(need, dtype=torch.uint8, device=dev)
+            d["do"] = torch.empty_like(d["dq"])
+            d["dlse"] = torch.empty((c.num_seqs, c.Hq), dtype=torch.float32, device=dev)
+
+    def second_buffer_set(self):
+        """Another set of per-step input and output buffers on the device; the
+        resident KV caches and the decode workspace are shared with the first."""
+        d = dict(self.dev)
+        for name in self.host:
+            d[name] = torch.empty_like(self.dev[name])
+        self._alloc_outputs(d)
+        return d
 
     def launches_per_step(self) -> int:
         return ((1 if self.prefill_cfg is not None else 0) + (2 if self.decode_cfg is not None else 0) +
@@ -358,30 +398,18 @@ class Step:
         self.api.attn_fwd(d["q"], d["k"], d["v"], c.causal, c.scale, out=d["o"], lse=d["lse"],
                           window_left=c.window_left if c.window_left >= 0 else None)
 
-    def run_decode(self, d=None):
+    def run_decode(self, d=None, graph=None):
         d = d or self.dev
-        if self.graph is not None:
-            self.graph.launch()
+        graph = graph if graph is not None else (self.graph if d is self.dev else None)
+        if graph is not None:
+            graph.launch()
             return
         c = self.decode_cfg
         self.api.paged_attn_decode(d["dq"], d["k_pool"], d["v_pool"], d["block_table"], d["seq_lens"], c.scale,
-                                   workspace=self.dev["ws"], out=d["do"], lse=d["dlse"])
-
-    def tensor_peak_tflops(self, peaks) -> float:
-        """Peak for this step's contraction dtype: the measured bf16 GEMM
-        rate, doubled for e4m3 (the nominal dense fp8 / bf16 ratio, 4.5 / 2.25
-        PFLOP/s)."""
-        return peaks["bf16_tflops"] * (2.0 if self.fp8 else 1.0)
-
-    def ideal_seconds(self, peaks) -> float:
-        """Separate kernels add up; within the prefill kernel the tensor work
-        and the bytes it moves overlap, so the slower of the two counts."""
-        prefill = max(self.flops / (self.tensor_peak_tflops(peaks) * 1e12),
-                      self.fused_bytes / (peaks["hbm_gbs"] * 1e9))
-        return prefill + self.bytes / (peaks["hbm_gbs"] * 1e9)
+                                   workspace=d["ws"], out=d["do"], lse=d["dlse"])
 
 
-def config_dict(step: Step, n_gpus: int):
+def config_dict(step: StepSpec, n_gpus: int, decode_graph: bool = False):
     cfg = {"workload": None, "parallelism": f"replicas{n_gpus}" if n_gpus > 1 else "single"}
     parts = []
     if step.prefill_cfg is not None:
@@ -411,7 +439,7 @@ def config_dict(step: Step, n_gpus: int):
                          "len_range": [c.min_len, c.max_len], "total_tokens": int(L.sum()),
                          "num_pages": step.decode_inp["num_pages"], "seed": c.seed, "bytes": step.bytes}
     cfg["workload"] = " + ".join(parts)
-    if step.graph is not None:
+    if decode_graph and step.decode_cfg is not None:
         cfg["decode_graph"] = True
     if step.decode_cfg is not None:
         cfg["l2"] = "inputs larger than L2: the decode pass streams >1 GB of KV through the 126 MB L2 every step"
@@ -553,7 +581,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     peaks = load_peaks()
-    step = StepHost(args.workload)
+    step = StepHost(args.workload, world, args.decode_graph)
     cfgs = (step.prefill_cfg, step.decode_cfg, step.host, step.decode_inp, step.chunked, step.fp8, step.mask)
     for _ in range(args.warmup):
         oracle_sample(cfgs, 0.0, per_call=True)
@@ -584,52 +612,84 @@ def run_reference(args, world, rank):
 
 
 class StepHost:
-    """Host-only inputs for the reference arm (no GPU needed)."""
+    """Host-only inputs for the reference arm (no GPU needed): the same
+    StepSpec as our arm (rank 0's draw), in the forms the oracle takes."""
 
-    def __init__(self, workload):
-        self.prefill_cfg = self.decode_cfg = None
-        self.host = {}
-        self.decode_inp = None
-        self.chunked = None
-        self.fp8 = None
-        self.mask = None
-        parts = []
-        if workload in FP8_WORKLOADS:
-            self.prefill_cfg = W.PREFILL_CONFIGS[FP8_WORKLOADS[workload]]
-            (q, k, v), self.fp8 = W.make_prefill_inputs_fp8(self.prefill_cfg)
-            self.host.update(q=q, k=k, v=v)
-            parts.append(prefill_label(self.prefill_cfg, True))
-        if workload in CHUNKED_WORKLOADS:
-            c = W.CHUNKED_CONFIGS[workload]
-            self.chunked = (c, W.make_chunked_inputs(c))
-            parts.append(chunked_label(c))
-        if workload in PREFILL_WORKLOADS:
-            name = "causal_mha" if workload == "default" else workload
-            self.prefill_cfg = W.PREFILL_CONFIGS[name]
-            q, k, v = W.make_prefill_inputs(self.prefill_cfg)
-            self.host.update(q=q, k=k, v=v)
-            parts.append(prefill_label(self.prefill_cfg))
-        if workload in MASK_WORKLOADS:
-            name, kind = MASK_WORKLOADS[workload]
-            c = self.prefill_cfg = W.PREFILL_CONFIGS[name]
-            q, k, v = W.make_prefill_inputs(c)
-            self.host.update(q=q, k=k, v=v)
-            self.mask = oracle_mask(kind, c)
-            parts.append(prefill_label(c, mask_kind=kind))
-        if workload in DECODE_WORKLOADS:
-            self.decode_cfg = W.DECODE_CONFIGS["small_decode" if workload == "small_decode" else "paged_decode"]
-            inp = W.make_decode_inputs(self.decode_cfg)
-            self.decode_inp = inp
-            self.host.update(dq=inp["q"], k_pool=inp["k_pool"], v_pool=inp["v_pool"],
-                             block_table=inp["block_table"], seq_lens=inp["seq_lens"])
-            c = self.decode_cfg
-            parts.append(f"paged decode {c.num_seqs} seqs Hq={c.Hq} Hkv={c.Hkv} d={c.d} page={c.page_size}")
-        self.config = {"workload": " + ".join(parts), "parallelism": "single"}
+    def __init__(self, workload, world: int = 1, decode_graph: bool = False):
+        spec = StepSpec(workload, 0, mask_tensors=False)  # the oracle builds M rows itself
+        self.prefill_cfg = spec.prefill_cfg
+        self.decode_cfg = spec.decode_cfg
+        self.host = {**spec.host, **spec.resident}
+        self.decode_inp = spec.decode_inp
+        self.chunked = (spec.chunked_cfg, spec.chunked_inp) if spec.chunked_cfg is not None else None
+        self.fp8 = spec.descales if spec.fp8 else None
+        self.mask = oracle_mask(spec.mask_kind, spec.prefill_cfg) if spec.mask_kind is not None else None
+        self.config = config_dict(spec, world, decode_graph)
 
 
 def unit_string() -> str:
     return ("fraction of B200 peak (time-weighted: prefill tensor FLOP/s at the inputs' dtype peak, "
             "decode/append HBM B/s), summed over GPUs")
+
+
+# The benchmark configurations the default step does not run (the step is the
+# causal MHA prefill + the paged decode), each timed on its own in the same
+# run: label, prefill config, e4m3 inputs.
+SWEEP = (("C1", "tiny", False), ("C3", "causal_gqa", False), ("C5", "long_causal", False),
+         ("C3 fp8", "causal_gqa", True), ("C5 fp8", "long_causal", True))
+
+
+def config_sweep(api, peaks, device, reps: int):
+    """Per-launch time of the prefill kernel on each SWEEP configuration:
+    CUDA events around each launch, a 256 MB L2 flush (written, then read
+    back) before each one, inputs resident.  The tiny C1 case is reported as
+    latency; the others as TFLOP/s against the bf16 peak (e4m3: twice it)."""
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    sink = torch.zeros((), dtype=torch.int64, device=device)
+    out = {}
+    for label, name, fp8 in SWEEP:
+        c = W.PREFILL_CONFIGS[name]
+        if fp8:
+            qkv, (qd, kd, vd) = W.make_prefill_inputs_fp8(c)
+        else:
+            qkv = W.make_prefill_inputs(c)
+        q, k, v = (x.to(device) for x in qkv)
+        o = torch.empty(q.shape, dtype=torch.bfloat16, device=device)
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=device)
+
+        def call():
+            if fp8:
+                api.attn_fwd_fp8(q, k, v, c.causal, c.scale, qd, kd, vd, out=o, lse=lse)
+            else:
+                api.attn_fwd(q, k, v, c.causal, c.scale, out=o, lse=lse)
+
+        for _ in range(3):
+            call()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        stream = torch.cuda.current_stream()
+        for a, b in evs:
+            flush.fill_(1)
+            sink.copy_(flush.view(torch.int64).sum())
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        times = [a.elapsed_time(b) / 1e3 for a, b in evs]
+        per = sum(times) / len(times)
+        flops = W.prefill_flops(c)
+        entry = {"config": f"{label} {prefill_label(c, fp8)}", "us_per_launch": per * 1e6,
+                 "us_min": min(times) * 1e6, "launches": reps, "algorithmic": flops}
+        if name == "tiny":
+            entry.update(bound="launch", unit="us", achieved=per * 1e6)
+        else:
+            tfl = flops / per / 1e12
+            tpk = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+            entry.update(bound="tensor", unit="TFLOP/s", achieved=tfl, peak=tpk, frac=tfl / tpk)
+        out[f"prefill_fwd_kernel {label}"] = entry
+        del q, k, v, o, lse
+    if api.device_status() != 0:
+        raise RuntimeError("a kernel reported a device error in the configuration sweep")
+    return out
 
 
 def run_ours(args, world, rank, local_rank):
@@ -715,7 +775,7 @@ def run_ours(args, world, rank, local_rank):
         "metric": METRIC, "value": value, "unit": unit_string(), "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * t_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if step.fp8 else "bf16", "data": "synthetic",
-        "config": config_dict(step, world),
+        "config": config_dict(step, world, args.decode_graph),
         "gpu_launches": step.launches_per_step() * args.steps,
         "clocks": clocks.summary(),
         "peaks": peaks,
@@ -755,7 +815,11 @@ def run_ours(args, world, rank, local_rank):
                                                  "us_per_launch": per * 1e6, "algorithmic": step.flops}
         line["prefill_tflops"] = tfl
         line["append_gbs"] = gbs
-    dominant = max(kernels, key=lambda k: kernels[k]["us_per_launch"])
+    dominant = max(kernels, key=lambda k: kernels[k]["us_per_launch"])  # of the step's own kernels
+    if args.workload == "default" and not args.no_sweep:
+        with ClockSampler(device) as sweep_clocks:
+            kernels.update(config_sweep(api, peaks, device, max(5, min(args.steps, 20))))
+        line["sweep_clocks"] = sweep_clocks.summary()
     traffic = load_traffic()
     dk = kernels[dominant]
     # Records are keyed by the bench workload whose launches ncu captured; the
@@ -795,45 +859,75 @@ def run_ours(args, world, rank, local_rank):
 
 def run_e2e(step: Step, args, world, device, peaks):
     """Same metric through the public API, host buffers: every step copies its
-    inputs from pinned host memory and reads the results back."""
+    inputs in from pinned host memory and reads its results back.  Two sets
+    of device buffers alternate, with the copies on their own streams, so a
+    step's upload and the previous step's download overlap the current
+    step's kernels, as a serving loop would run them; each step still moves
+    all of its own bytes."""
     pinned = {n: t.pin_memory() for n, t in step.host.items()}
-    outs = {}
-    for n in ("o", "lse", "do", "dlse", "co", "clse"):
-        if n in step.dev:
-            outs[n] = torch.empty(step.dev[n].shape, dtype=step.dev[n].dtype, pin_memory=True)
+    out_names = [n for n in Step.OUTPUTS if n in step.dev]
+    sets = [step.dev, step.second_buffer_set()]
+    graphs = [step.graph, step.make_graph(sets[1]) if step.graph is not None else None]
+    host_out = [{n: torch.empty(step.dev[n].shape, dtype=step.dev[n].dtype, pin_memory=True) for n in out_names}
+                for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values())
-    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
     steps = max(1, min(args.steps, args.e2e_steps))
-    stream = torch.cuda.current_stream()
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
 
-    def one():
-        for n, t in pinned.items():
-            step.dev[n].copy_(t, non_blocking=True)
+    def one(i):
+        b = i % 2
+        d = sets[b]
+        with torch.cuda.stream(up):
+            if i >= 2:
+                up.wait_event(computed[b])  # step i-2 has read this set's inputs
+            for n, t in pinned.items():
+                d[n].copy_(t, non_blocking=True)
+            uploaded[b].record(up)
+        comp.wait_event(uploaded[b])
+        if i >= 2:
+            comp.wait_event(downloaded[b])  # step i-2's results have left this set's outputs
         if step.prefill_cfg is not None:
-            step.run_prefill()
+            step.run_prefill(d)
         if step.decode_cfg is not None:
-            step.run_decode()
+            step.run_decode(d, graphs[b])
         if step.chunked_cfg is not None:
-            step.run_chunked(one_call=True)
-        for n, t in outs.items():
-            t.copy_(step.dev[n], non_blocking=True)
+            step.run_chunked(d, one_call=True)
+        computed[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(computed[b])
+            for n, t in host_out[b].items():
+                t.copy_(d[n], non_blocking=True)
+            downloaded[b].record(down)
 
-    one()
+    def drain():
+        comp.wait_event(downloaded[0])
+        comp.wait_event(downloaded[1])
+
+    for i in range(2):  # warm both buffer sets
+        one(i)
+    drain()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    a.record(stream)
-    for _ in range(steps):
-        one()
-    b.record(stream)
+    a.record(comp)
+    up.wait_event(a)
+    for i in range(steps):
+        one(i)
+    drain()
+    b.record(comp)
     torch.cuda.synchronize()
     secs = max_over_ranks(a.elapsed_time(b) / 1e3, world, device)
     ideal = sum_over_ranks(step.ideal_seconds(peaks) * steps, world, device)
     return {"value": ideal / secs, "unit": unit_string(), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": steps, "ms_per_step": 1e3 * secs / steps}
+            "steps": steps, "ms_per_step": 1e3 * secs / steps, "buffers": "double (copy streams overlap kernels)"}
 
 
 def main(argv=None):
@@ -850,6 +944,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip timing the other benchmark configurations (default workload only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

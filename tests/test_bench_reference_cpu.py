@@ -27,6 +27,9 @@ def test_reference_arm_line(workload):
     assert line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"]
+    # the same config object as our arm reports for this workload (one GPU)
+    import bench
+    assert line["config"] == json.loads(json.dumps(bench.config_dict(bench.StepSpec(workload, mask_tensors=False), 1)))
     if workload != "tiny":
         assert "mask" in line["config"]["workload"] or "M per head" in line["config"]["workload"]
 

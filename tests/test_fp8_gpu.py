@@ -102,6 +102,19 @@ def test_fp8_causal_gqa_full_size_sampled():
     check(cfg, rows=[0, 1, 127, 128, 4095, 8190, 8191], heads=[(0, 0), (0, 5), (0, 31)])
 
 
+def test_fp8_long_causal_full_size_sampled():
+    """The benchmarked e4m3 long-context workload at full size (N = 32768, a
+    per-key K offset with sigma 2): work items of up to 256 KV tiles, where
+    the running max rises past the 0.5 lazy-rescale limit again and again and
+    most weights fall deep into the e4m3 subnormal range.  Fixed rows at the
+    start, the middle and the end of the sequence plus seeded random rows, on
+    the first and last head."""
+    cfg = W.PREFILL_CONFIGS["long_causal"]
+    rng = np.random.default_rng(5)
+    rows = sorted(set([0, 1, 128, 16383, 32766, 32767] + rng.integers(0, cfg.N, 6).tolist()))
+    check(cfg, rows=rows, heads=[(0, 0), (0, 7)])
+
+
 def test_fp8_descales_scale_the_result():
     """Doubling the V descale doubles O (bit for bit in fp32 before the bf16
     rounding, and bf16 doubling is exact); Q/K descales act through the
