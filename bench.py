@@ -120,7 +120,11 @@ def sum_over_ranks(x: float, world: int, device=None) -> float:
 
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML while running."""
+    """Samples the SM clock and clock-event reasons through NVML on a thread
+    that runs from construction until close(); every sample carries its host
+    time, so a region's samples are the ones taken inside its window (an NVML
+    call takes about a millisecond: a thread started only at the region's
+    start saw one sample of a 6 ms region)."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -128,9 +132,9 @@ class ClockSampler:
         0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, device, period_s: float = 0.001):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
-        self.period = period_s
+    def __init__(self, device):
+        self.samples = []  # (host time, SM MHz, reason bits)
+        self.max_mhz = None
         self._stop = threading.Event()
         self._thread = None
         try:
@@ -145,35 +149,43 @@ class ClockSampler:
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
         except Exception:  # NVML missing: report no samples
             self._nvml = None
+            return
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
 
     def _run(self):
         n = self._nvml
         while not self._stop.is_set():
             try:
-                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                mhz = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
                 bits = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for b, name in self.REASONS.items():
-                    if bits & b and name != "gpu_idle":
-                        self.reasons.add(name)
+                self.samples.append((time.perf_counter(), mhz, bits))
             except Exception:
                 pass
-            time.sleep(self.period)
+            time.sleep(0.0002)
 
-    def __enter__(self):
-        if self._nvml is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
-        return self
-
-    def __exit__(self, *exc):
+    def close(self):
         self._stop.set()
         if self._thread is not None:
             self._thread.join()
+            self._thread = None
 
-    def summary(self):
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
-                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples)}
+    def window(self, t0: float, t1: float, edge_s: float = 0.02):
+        """Summary of the samples taken between host times t0 and t1, plus the
+        nearest sample on each side when it lies within edge_s of the window
+        (so a region shorter than one NVML call still has the clock it ran at)."""
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        before = [s for s in self.samples if t0 - edge_s <= s[0] < t0][-1:]
+        after = [s for s in self.samples if t1 < s[0] <= t1 + edge_s][:1]
+        use = before + inside + after
+        reasons = set()
+        for _, _, bits in use:
+            for b, name in self.REASONS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in use) if use else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(inside), "samples_with_neighbours": len(use)}
 
 
 # ----------------------------------------------------------------------------- workload
@@ -727,6 +739,15 @@ def run_ours(args, world, rank, local_rank):
             flush.fill_(1)
             flush_sink.copy_(flush.view(torch.int64).sum())
 
+    clocks = ClockSampler(device)  # samples from here on; the timed regions pick their windows
+    try:
+        return _timed(args, world, rank, device, peaks, api, step, stream, one_step, clocks, flush)
+    finally:
+        clocks.close()
+
+
+def _timed(args, world, rank, device, peaks, api, step, stream, one_step, clocks, flush):
+    """Warm-up, the timed steps, the end-to-end leg, the sweep and the JSON line."""
     for _ in range(args.warmup):
         one_step()
     if api.device_status() != 0:
@@ -739,12 +760,13 @@ def run_ours(args, world, rank, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(device) as clocks:
-        start.record(stream)
-        for i in range(args.steps):
-            one_step(evs[i])
-        end.record(stream)
-        torch.cuda.synchronize()
+    t_host0 = time.perf_counter()
+    start.record(stream)
+    for i in range(args.steps):
+        one_step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
     if world > 1:
         torch.distributed.barrier()
     if api.device_status() != 0:
@@ -777,7 +799,7 @@ def run_ours(args, world, rank, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3" if step.fp8 else "bf16", "data": "synthetic",
         "config": config_dict(step, world, args.decode_graph),
         "gpu_launches": step.launches_per_step() * args.steps,
-        "clocks": clocks.summary(),
+        "clocks": clocks.window(t_host0, t_host1),
         "peaks": peaks,
     }
     kernels = {}
@@ -817,9 +839,9 @@ def run_ours(args, world, rank, local_rank):
         line["append_gbs"] = gbs
     dominant = max(kernels, key=lambda k: kernels[k]["us_per_launch"])  # of the step's own kernels
     if args.workload == "default" and not args.no_sweep:
-        with ClockSampler(device) as sweep_clocks:
-            kernels.update(config_sweep(api, peaks, device, max(5, min(args.steps, 20))))
-        line["sweep_clocks"] = sweep_clocks.summary()
+        t_sweep0 = time.perf_counter()
+        kernels.update(config_sweep(api, peaks, device, max(5, min(args.steps, 20))))
+        line["sweep_clocks"] = clocks.window(t_sweep0, time.perf_counter())
     traffic = load_traffic()
     dk = kernels[dominant]
     # Records are keyed by the bench workload whose launches ncu captured; the

@@ -194,3 +194,21 @@ def test_traffic_records_follow_each_kernels_sources(tmp_path, monkeypatch):
     # every kernel the bench reports has a source set, and every listed file exists
     for k, files in bench.KERNEL_SOURCE_SETS.items():
         assert set(files) <= set(bench.KERNEL_SOURCES)
+
+
+def test_clock_window_picks_the_samples_of_a_region():
+    """bench.ClockSampler.window: the samples inside the host-time window plus
+    the nearest one on each side if it lies within 20 ms; reasons from those
+    samples only."""
+    import bench
+    s = object.__new__(bench.ClockSampler)
+    s.max_mhz = 1965
+    ms = 1e-3
+    s.samples = [(0.0, 1000, 0x1), (10 * ms, 1965, 0x0), (11 * ms, 1965, 0x4), (12 * ms, 1800, 0x0),
+                 (30 * ms, 1965, 0x0), (900 * ms, 500, 0x40)]
+    w = s.window(10.5 * ms, 12.5 * ms)
+    assert w["samples"] == 2 and w["samples_with_neighbours"] == 4   # 10 ms and 30 ms are neighbours
+    assert w["sm_mhz"] == 1965 and w["reasons"] == ["sw_power_cap"]  # 0x40 at 900 ms is too far away
+    short = s.window(11.2 * ms, 11.3 * ms)                            # shorter than one sample period
+    assert short["samples"] == 0 and short["samples_with_neighbours"] == 2 and short["sm_mhz"] == 1882.5
+    assert s.window(500 * ms, 600 * ms)["sm_mhz"] is None              # nothing near
