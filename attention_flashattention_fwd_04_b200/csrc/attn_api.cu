@@ -177,8 +177,9 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const attn::Deco
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail_cuda(e);
   const long long warps = static_cast<long long>(p.S) * p.Hq;
-  const unsigned mgrid = static_cast<unsigned>((warps * 32 + 255) / 256);
-  attn::decode_merge_kernel<D><<<mgrid, 256, 0, stream>>>(p, reinterpret_cast<__nv_bfloat16*>(o), lse);
+  const unsigned mgrid = static_cast<unsigned>((warps * 32 + attn::kMergeThreads - 1) / attn::kMergeThreads);
+  attn::decode_merge_kernel<D><<<mgrid, attn::kMergeThreads, 0, stream>>>(p, reinterpret_cast<__nv_bfloat16*>(o),
+                                                                           lse);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail_cuda(e);
   return ATTN_OK;

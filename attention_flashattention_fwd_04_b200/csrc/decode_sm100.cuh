@@ -323,10 +323,14 @@ __global__ void __launch_bounds__(32 * (HB + 1), 1)
 }
 
 // One warp per (sequence, query head): combine the splits that hold tokens.
-// Lane i computes the weight of split i of each group of 32; the partial rows
-// are then read eight splits at a time so that eight loads are in flight.
+// Lane i computes the weight of split i of each group of 32.  Up to 32
+// splits, every partial row is requested together with the partial LSEs (the
+// rows do not depend on the weights), so the merge costs two dependent trips
+// to memory (the length, then everything); longer sequences read the rows 16
+// splits per round after the weights.
+constexpr int kMergeThreads = 128;
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kMergeThreads)
     decode_merge_kernel(const DecodeParams p, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -345,6 +349,48 @@ __global__ void __launch_bounds__(256)
   const float* plse = p.part_lse + static_cast<size_t>(wid) * p.max_splits;
   const float* po = p.part_o + static_cast<size_t>(wid) * p.max_splits * D + lane * kPer;
   constexpr float kLog2e = 1.4426950408889634f;
+  if (n_splits <= 32) {
+    const float pl = lane < n_splits ? plse[lane] : -INFINITY;
+    float v[32][kPer];
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      if (u < n_splits) {
+        const float* src = po + static_cast<size_t>(u) * D;
+        if constexpr (kPer == 4) {
+          const float4 x = *reinterpret_cast<const float4*>(src);
+          v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+        } else {
+          const float2 x = *reinterpret_cast<const float2*>(src);
+          v[u][0] = x.x; v[u][1] = x.y;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) v[u][e] = 0.f;
+      }
+    }
+    float mx = pl;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const float my_w = lane < n_splits ? ex2_approx((pl - mx) * kLog2e) : 0.f;
+    float wsum = my_w;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+    float out[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) out[e] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const float w = __shfl_sync(0xffffffffu, my_w, u);
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) out[e] = fmaf(w, v[u][e], out[e]);
+    }
+    const float inv = 1.f / wsum;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2)
+      *reinterpret_cast<uint32_t*>(orow + lane * kPer + e) = pack_bf16x2(out[e] * inv, out[e + 1] * inv);
+    if (lane == 0) lse[wid] = mx + logf(wsum);
+    return;
+  }
   // The first 32 splits' LSEs stay in registers (lane t: split t) for the
   // weights; the partial rows are then read 16 splits per round, so a
   // sequence of up to 32 splits costs three dependent trips to memory.
