@@ -704,6 +704,42 @@ def config_sweep(api, peaks, device, reps: int):
     return out
 
 
+def sdpa_context(peaks, device, reps: int):
+    """Context, not a target: PyTorch's own scaled_dot_product_attention
+    (default backend) on the C2, C3 and C5 inputs, timed as config_sweep
+    times ours (events around each call, the 256 MB L2 flush before it)."""
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    sink = torch.zeros((), dtype=torch.int64, device=device)
+    out = {}
+    for label, name in (("C2", "causal_mha"), ("C3", "causal_gqa"), ("C5", "long_causal")):
+        c = W.PREFILL_CONFIGS[name]
+        q, k, v = (x.to(device) for x in W.make_prefill_inputs(c))
+
+        def call():
+            return torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=c.causal, scale=c.scale,
+                                                                    enable_gqa=c.Hq != c.Hkv)
+
+        for _ in range(3):
+            call()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        stream = torch.cuda.current_stream()
+        for a, b in evs:
+            flush.fill_(1)
+            sink.copy_(flush.view(torch.int64).sum())
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+        times = [a.elapsed_time(b) / 1e3 for a, b in evs]
+        per = sum(times) / len(times)
+        tfl = W.prefill_flops(c) / per / 1e12
+        out[f"torch_sdpa {label}"] = {"config": f"{label} {prefill_label(c, False)}", "us_per_launch": per * 1e6,
+                                      "us_min": min(times) * 1e6, "unit": "TFLOP/s", "achieved": tfl,
+                                      "frac": tfl / peaks["bf16_tflops"]}
+        del q, k, v
+    return out
+
+
 def run_ours(args, world, rank, local_rank):
     from attention_flashattention_fwd_04_b200 import api
     from attention_flashattention_fwd_04_b200.build import build
@@ -841,6 +877,7 @@ def _timed(args, world, rank, device, peaks, api, step, stream, one_step, clocks
     if args.workload == "default" and not args.no_sweep:
         t_sweep0 = time.perf_counter()
         kernels.update(config_sweep(api, peaks, device, max(5, min(args.steps, 20))))
+        line["context"] = sdpa_context(peaks, device, max(5, min(args.steps, 20)))
         line["sweep_clocks"] = clocks.window(t_sweep0, time.perf_counter())
     traffic = load_traffic()
     dk = kernels[dominant]
