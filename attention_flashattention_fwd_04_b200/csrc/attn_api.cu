@@ -178,8 +178,20 @@ int launch_decode(const CUtensorMap& tk, const CUtensorMap& tv, const attn::Deco
   if (e != cudaSuccess) return fail_cuda(e);
   const long long warps = static_cast<long long>(p.S) * p.Hq;
   const unsigned mgrid = static_cast<unsigned>((warps * 32 + attn::kMergeThreads - 1) / attn::kMergeThreads);
-  attn::decode_merge_kernel<D><<<mgrid, attn::kMergeThreads, 0, stream>>>(p, reinterpret_cast<__nv_bfloat16*>(o),
-                                                                           lse);
+  // The merge may launch while the split pass's last wave runs (see
+  // decode_split_kernel); it waits for the split grid in griddepcontrol.wait.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(mgrid);
+  cfg.blockDim = dim3(attn::kMergeThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, attn::decode_merge_kernel<D>, p, reinterpret_cast<__nv_bfloat16*>(o), lse);
+  if (e != cudaSuccess) return fail_cuda(e);
   e = cudaGetLastError();
   if (e != cudaSuccess) return fail_cuda(e);
   return ATTN_OK;

@@ -96,6 +96,11 @@ __global__ void __launch_bounds__(32 * (HB + 1), 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using L = DecodeLayout<D, HB>;
+  // The merge grid (launched as a programmatic dependent) may start once every
+  // CTA of this grid has started: it then waits for this grid's completion in
+  // griddepcontrol.wait, so its launch overlaps this grid's last wave.  All
+  // split CTAs are resident or done by then, so none waits for an SM.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int split = blockIdx.x;
   const int s = blockIdx.y;
   const int head0 = blockIdx.z * HB;  // first kv head of this CTA
@@ -332,6 +337,10 @@ constexpr int kMergeThreads = 128;
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads)
     decode_merge_kernel(const DecodeParams p, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+  // Launched as a programmatic dependent of the split pass: wait until that
+  // grid has completed and its partials are visible (returns at once when
+  // launched without the attribute).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= p.S * p.Hq) return;
