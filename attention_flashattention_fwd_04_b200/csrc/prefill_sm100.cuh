@@ -1203,6 +1203,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mb[v] = make_uint4(0u, 0u, 0u, 0u);
             if (grow < p.N && kv0 + 8 * v < p.N) mb[v] = __ldg(reinterpret_cast<const uint4*>(brow) + v);
           }
+          // The next tile's 256 bytes of this row into L2 (two lines), one step
+          // before they are loaded; only bytes that load reads.  (Two or three
+          // steps ahead measured slower, and bulk prefetches from the producer
+          // warp clogged the copy engine that brings K and V.)
+          if (!SPARSE && grow < p.N && jj + 1 < n_t) {
+            const int kv1 = kv0 + 128;
+            const char* nxt = reinterpret_cast<const char*>(brow + 128);
+            if (kv1 < p.N) prefetch_l2(nxt);
+            if (kv1 + 64 < p.N) prefetch_l2(nxt + 128);
+          }
         }
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarSFull + t), s_cnt++ & 1u, kErrWaitSFull));
         if (!ok) break;
